@@ -1,0 +1,496 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged KV-cache decode step on B200.
+
+One step = the whole hot path over one batch: kv_cache_write of every
+sequence's newest token through slot_mapping, then paged_attention_decode of
+one query token per sequence over its paged KV cache (plus the log-sum-exp
+merge when the plan splits the context).  Inputs are seeded synthetic data of
+the workload's shapes and distributions, resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py --impl reference ...      # the fp64 CPU oracle, timed on host cores
+
+Multi-GPU (launched by torch.distributed.run): every rank runs an independent
+replica of the workload on its own GPU (the path shards by sequence with no
+exchange step); the job time is the max over ranks and `value` counts the
+bytes of all ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_468_b200 import workloads  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s (fraction of B200 HBM peak); decode tokens/s"
+KERNEL_SOURCES = ["paged_kv_cache_468_b200/csrc/pkv_kernels.cuh",
+                  "paged_kv_cache_468_b200/csrc/pkv_ptx.cuh",
+                  "paged_kv_cache_468_b200/csrc/pagedkv.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- helpers --
+
+def esize(dtype: str) -> int:
+    return 2
+
+
+def step_bytes(step: dict, cfg: workloads.DecodeConfig) -> dict:
+    """Algorithmic bytes of one step (each byte the definition must touch once)."""
+    lens = [int(x) for x in step["context_lens"]]
+    B, Hq, D = step["query"].shape
+    Hkv, bs, es = cfg.num_kv_heads, cfg.block_size, esize(cfg.dtype)
+    kv = sum(lens) * Hkv * D * es * 2                         # K and V rows, read once
+    qo = 2 * B * Hq * D * es                                  # query read + output written
+    tables = 4 * (sum(-(-L // bs) for L in lens) + B)         # used table entries + lengths
+    decode = kv + qo + tables
+    T = int((step["slot_mapping"] >= 0).sum())
+    write = 2 * (2 * T * Hkv * D * es) + 8 * T                # K,V rows read+written, slots
+    # shared prefix: unique KV bytes (each shared block counted once)
+    uniq_rows = 0
+    seen = set()
+    for b, L in enumerate(lens):
+        nblk = -(-L // bs)
+        for i in range(nblk):
+            blk = int(step["block_tables"][b, i])
+            if blk in seen:
+                continue
+            seen.add(blk)
+            uniq_rows += min(bs, L - i * bs)
+    kv_unique = uniq_rows * Hkv * D * es * 2
+    return dict(kv=kv, kv_unique=kv_unique, decode=decode,
+                decode_unique=decode - kv + kv_unique, write=write,
+                tokens=B, kv_tokens=sum(lens))
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(config_name: str):
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel sources and this workload (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = d.get(config_name)
+    if not entry or entry.get("source_sha") != kernel_source_sha():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+        self.t_on = None
+        self.t_off = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        t0 = time.time()
+        while not self.lines and time.time() - t0 < 5:
+            time.sleep(0.02)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, on: bool):
+        if on:
+            self.t_on = time.time()
+        else:
+            self.t_off = time.time()
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for t, line in self.lines:
+            if self.t_on is not None and self.t_off is not None and not (self.t_on <= t <= self.t_off + 0.06):
+                continue
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            rows.append(parts)
+        if not rows:   # timed region shorter than the sampling period: take the nearest
+            rows = [[p.strip() for p in l.split(",")] for _, l in self.lines[-3:]]
+            rows = [r for r in rows if len(r) == len(self.FIELDS)]
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ------------------------------------------------------- CPU oracle timing --
+
+def oracle_sample_rate(step: dict, cfg, seconds: float, nthreads: int, max_seqs=None):
+    """Run the fp64 oracle (write + decode) on the first sequences of the step
+    until `seconds` pass; returns (GB/s, sample description, threads)."""
+    import numpy as np
+    import oracle
+
+    def u16(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    B = step["query"].shape[0]
+    n = B if max_seqs is None else max(1, min(B, max_seqs))
+    q = u16(step["query"][:n])
+    kc = u16(step["key_cache"]).copy()
+    vc = u16(step["value_cache"]).copy()
+    bt = step["block_tables"][:n].numpy()
+    cl = step["context_lens"][:n].numpy()
+    nk, nv = u16(step["new_key"][:n]), u16(step["new_value"][:n])
+    slots = step["slot_mapping"][:n].numpy()
+    sub = dict(step, query=step["query"][:n], context_lens=step["context_lens"][:n],
+               block_tables=step["block_tables"][:n], slot_mapping=step["slot_mapping"][:n])
+    nbytes = step_bytes(sub, cfg)
+    per = nbytes["decode"] + nbytes["write"]
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle.kv_cache_write(nk, nv, slots, kc, vc, cfg.block_size)
+        oracle.paged_attention_decode(q, kc, vc, bt, cl, cfg.scale, cfg.dtype, nthreads=nthreads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return per * reps / el / 1e9, n, reps, el
+
+
+def choose_oracle_seqs(step, cfg, nthreads, budget_s):
+    """Largest prefix of the batch whose oracle step fits in budget_s."""
+    _, _, _, el = oracle_sample_rate(step, cfg, 0.0, nthreads, max_seqs=1)
+    B = step["query"].shape[0]
+    return max(1, min(B, int(budget_s / max(el, 1e-6))))
+
+
+def run_reference(args, cfg, world, rank):
+    """The oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return 0
+    nthreads = os.cpu_count() or 1
+    step = workloads.make_decode_step(cfg)
+    total_budget = args.reference_seconds
+    per_step = total_budget / max(1, args.steps + args.warmup)
+    nseq = choose_oracle_seqs(step, cfg, nthreads, per_step)
+    for _ in range(args.warmup):
+        oracle_sample_rate(step, cfg, 0.0, nthreads, max_seqs=nseq)
+    t_total, gbs_bytes = 0.0, 0.0
+    for _ in range(args.steps):
+        gbs, n, reps, el = oracle_sample_rate(step, cfg, 0.0, nthreads, max_seqs=nseq)
+        t_total += el
+        gbs_bytes += gbs * el
+    value = gbs_bytes / t_total
+    sample = (f"first {nseq} of {cfg.batch} sequences per step (write + decode), "
+              f"{args.steps} timed steps, fp64 oracle")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": cfg.name, "description": cfg.description},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------- GPU arm ----
+
+def run_gpu(args, cfg, world, rank, local):
+    import paged_kv_cache_468_b200 as pkv
+
+    dev = torch.device("cuda", local)
+    step = workloads.make_decode_step(dataclass_replace(cfg, seed=cfg.seed + 1000 * rank))
+    nbytes = step_bytes(step, cfg)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
+    B, Hq, D = d["query"].shape
+    NB, bs, Hkv, _ = d["key_cache"].shape
+    MB = d["block_tables"].shape[1]
+    pt_req = cfg.partition_tokens if args.partition_tokens is None else args.partition_tokens
+    plan_pt, plan_np = pkv.decode_plan(B, Hq, Hkv, D, MB, bs, pt_req)
+    ws_bytes = pkv.decode_workspace_bytes(B, Hq, Hkv, D, MB, bs, pt_req)
+    ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(d["query"])
+    launches_per_step = 2 + (1 if plan_np > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+
+    def one_step():
+        pkv.kv_cache_write(d["new_key"], d["new_value"], d["slot_mapping"], d["key_cache"],
+                           d["value_cache"])
+        pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
+                                   d["context_lens"], d["scale"], partition_tokens=pt_req,
+                                   out=out, workspace=ws)
+
+    pkv.device_flags(clear=True)
+    for _ in range(args.warmup):
+        one_step()
+    torch.cuda.synchronize()
+
+    # ---- device-timed region (inputs resident in HBM) ----
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
+    if sampler:
+        sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    if sampler:
+        sampler.mark(True)
+    t_start.record(stream)
+    for i in range(K):
+        pkv.kv_cache_write(d["new_key"], d["new_value"], d["slot_mapping"], d["key_cache"],
+                           d["value_cache"])
+        ev[i][0].record(stream)
+        pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
+                                   d["context_lens"], d["scale"], partition_tokens=pt_req,
+                                   out=out, workspace=ws)
+        ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark(False)
+    barrier(world)
+    ms_total = t_start.elapsed_time(t_end)
+    ms_total_max = max_over_ranks(ms_total, world)
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)   # decode (+ merge) per launch
+    clocks = sampler.stop() if sampler else None
+    flags = pkv.device_flags(clear=True)
+
+    # ---- end to end through the public API, host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        host_in = {k: d[k].cpu().pin_memory() for k in
+                   ("query", "new_key", "new_value", "slot_mapping", "block_tables", "context_lens")}
+        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        d2h = host_out.numel() * host_out.element_size()
+        dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+
+        def e2e_step():
+            for k, v in host_in.items():
+                dev_in[k].copy_(v, non_blocking=True)
+            pkv.kv_cache_write(dev_in["new_key"], dev_in["new_value"], dev_in["slot_mapping"],
+                               d["key_cache"], d["value_cache"])
+            pkv.paged_attention_decode(dev_in["query"], d["key_cache"], d["value_cache"],
+                                       dev_in["block_tables"], dev_in["context_lens"], d["scale"],
+                                       partition_tokens=pt_req, out=out, workspace=ws)
+            host_out.copy_(out, non_blocking=True)
+            stream.synchronize()                       # the caller reads the result
+
+        for _ in range(max(3, args.warmup)):
+            e2e_step()
+        Ke = max(1, min(K, args.e2e_steps))
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(Ke):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
+        e2e_gbs = sum_over_ranks(nbytes["decode"] + nbytes["write"], world) / (e2e_ms * 1e-3) / 1e9
+        e2e = {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": Ke,
+               "tokens_per_s": round(sum_over_ranks(B, world) / (e2e_ms * 1e-3), 1)}
+
+    ms_step = ms_total_max / K
+    total_bytes = sum_over_ranks(nbytes["decode"] + nbytes["write"], world)
+    value = total_bytes / (ms_step * 1e-3) / 1e9
+    tokens = sum_over_ranks(B, world)
+
+    peaks = measured_peaks()
+    achieved = nbytes["decode_unique"] / (decode_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": committed_traffic(cfg.name),
+                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
+                if peaks["source"] == "measured" else "fallback 6650 GB/s",
+                "kernel": "paged_decode_kernel" + (" + lse_merge_kernel" if plan_np > 1 else ""),
+                "bytes_per_launch": nbytes["decode_unique"], "launch_ms": round(decode_ms, 5),
+                "frac_of_8000": round(achieved / 8000.0, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nthreads = os.cpu_count() or 1
+        nseq = choose_oracle_seqs(step, cfg, nthreads, args.cpu_seconds / 3)
+        gbs, n, reps, el = oracle_sample_rate(step, cfg, args.cpu_seconds, nthreads, max_seqs=nseq)
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+               "sample": f"first {n} of {B} sequences (write + decode), {reps} repetitions "
+                         f"in {el:.1f} s, fp64"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "description": cfg.description, "batch": B,
+                       "num_heads": Hq, "num_kv_heads": Hkv, "head_dim": D, "block_size": bs,
+                       "num_blocks": NB, "max_blocks": MB,
+                       "context_tokens": nbytes["kv_tokens"],
+                       "partition_tokens": plan_pt, "num_partitions": plan_np,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": (f"inputs larger than L2: {nbytes['kv_unique'] / 1e6:.0f} MB of K/V "
+                              f"per step vs 126 MB L2, no flush")
+                       if nbytes["kv_unique"] > 126e6 else "inputs fit in L2 (no flush)"},
+            "tokens_per_s": round(tokens / (ms_step * 1e-3), 1),
+            "kv_tokens_per_s": round(sum_over_ranks(nbytes["kv_tokens"], world) / (ms_step * 1e-3), 1),
+            "frac_of_hbm_peak": round(value / peaks["hbm_gbs"], 4),
+            "logical_kv_gbs": round(sum_over_ranks(nbytes["kv"], world) / (ms_step * 1e-3) / 1e9, 1),
+            "gpu_launches": launches_per_step * K,
+            "device_flags": flags,
+            "roofline": roofline,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def dataclass_replace(cfg, **kw):
+    import dataclasses
+    return dataclasses.replace(cfg, **kw)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--config", default=workloads.HEADLINE, choices=sorted(workloads.CONFIGS))
+    ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
+    ap.add_argument("--partition-tokens", type=int, default=None,
+                    help="override the workload's partition request (0 auto, <0 never)")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    cfg = workloads.CONFIGS[args.config]
+
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, cfg, world, rank)
+
+    world, rank, local = dist_setup()
+    if world != args.gpus and rank == 0:
+        print(f"note: --gpus {args.gpus} but WORLD_SIZE {world}; using {world}", file=sys.stderr)
+    try:
+        return run_gpu(args, cfg, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

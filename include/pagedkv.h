@@ -1,0 +1,217 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: paged KV-cache write and decode
+ * attention on NVIDIA B200 (sm_100a), plus the host block allocator that
+ * builds block tables.
+ *
+ * Sources (web pages describing vLLM's paged KV cache):
+ *   [YK] "大模型推理框架 vLLM 源码解析 一" (ai.yueke.cloud), section 三
+ *        "vLLM 源码关键路径解析": the cache shape
+ *        [num_blocks, block_size, num_heads, head_dim]; paged_attention_v1
+ *        takes (query, key_cache, value_cache, block_tables, context_lens);
+ *        for token j of sequence i the physical block is
+ *        block_tables[i][j // block_size] and the in-block offset is
+ *        j % block_size.  Section 二: BlockAllocator.allocate() returns a
+ *        list of physical block ids.  Section 四 step 4: --block-size
+ *        defaults to 16; 32 reduces block-table lookups.
+ *   [FC] "23.1 vLLM：高吞吐推理框架原理与部署" (r.flycode100.com), section 二
+ *        "PagedAttention 的核心原理": parts 1-2 (fixed blocks of 16 tokens,
+ *        one block allocated on arrival and one more every 16 tokens, a
+ *        block table keeps the logical order, blocks return to a shared free
+ *        pool when the request ends) and part 3 (prefix blocks are shared
+ *        between parallel samples / beams and copied only when a sequence
+ *        writes into a shared block: copy-on-write).
+ *   [MH] "大模型推理框架VLLM-0.7.3源码" (mhpq.cn), sections 2.1 and 3.3: the
+ *        model runner builds block_tables and slot_mapping; slot_mapping
+ *        tells the operator into which cell each current token's K/V goes.
+ *
+ * Conventions for every call below:
+ *   - Device pointers are caller-owned (the library never allocates or frees
+ *     device memory and never synchronises the device inside compute calls).
+ *     Tensors are dense and row-major in the shapes given; K/V/query/output
+ *     pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Compute calls are asynchronous on it.  The returned status
+ *     covers host-side validation and the launch; errors found while the
+ *     kernels run (a slot, block id or context length outside its range,
+ *     or a bounded wait that expired) set bits in a per-device flag word read
+ *     by pkv_device_flags().  Kernels never trap.
+ *   - Element types: PKV_F16 (IEEE binary16) or PKV_BF16 (bfloat16); the
+ *     query, caches and output share one type.  Scores, softmax and
+ *     accumulation are fp32; the output is rounded to nearest even.
+ *   - Supported shapes: head_dim in {64, 128}; block_size in {16, 32};
+ *     num_heads % num_kv_heads == 0 with group size 1..8;
+ *     num_blocks * block_size < 2^31.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,   /* null pointer, negative or inconsistent size */
+    PKV_ERR_UNSUPPORTED = 2,   /* shape outside the compiled set (see above) */
+    PKV_ERR_OUT_OF_RANGE = 3,  /* a host-visible index outside its pool */
+    PKV_ERR_OOM = 4,           /* allocator: not enough free blocks (nothing taken) */
+    PKV_ERR_CUDA = 5,          /* a CUDA runtime call failed; see pkv_last_error() */
+    PKV_ERR_WORKSPACE = 6,     /* workspace missing or smaller than required */
+    PKV_ERR_MISALIGNED = 7     /* a pointer is not 16-byte aligned */
+} pkv_status;
+
+typedef enum { PKV_F16 = 0, PKV_BF16 = 1 } pkv_dtype;
+
+/* Device flag bits (pkv_device_flags). */
+#define PKV_DEVFLAG_SLOT_RANGE    0x1u  /* write: slot >= num_blocks*block_size (token skipped) */
+#define PKV_DEVFLAG_BLOCK_RANGE   0x2u  /* decode: table entry outside [0, num_blocks) (block 0 read instead) */
+#define PKV_DEVFLAG_CONTEXT_RANGE 0x4u  /* decode: context_len < 0 or > max_blocks*block_size (clamped) */
+#define PKV_DEVFLAG_WAIT_TIMEOUT  0x8u  /* decode: a shared-memory pipeline wait gave up (output invalid) */
+
+/* Human-readable name of a status code (static string). */
+const char *pkv_status_str(pkv_status s);
+
+/* Detail of the last failing call on this host thread ("" if none). */
+const char *pkv_last_error(void);
+
+/* Library version string, e.g. "pagedkv 0.1.0 sm_100a". */
+const char *pkv_version(void);
+
+/*
+ * Read (and with clear != 0, reset) the device flag word of `device`.
+ * Synchronous: waits for all prior work on that device.
+ */
+pkv_status pkv_device_flags(int device, unsigned int *flags, int clear);
+
+/*
+ * kv_cache_write -- store the current tokens' K/V into their cache cells
+ * ([MH] 2.1, 3.3; cache shape [YK] 三).
+ *
+ *   key, value     [num_tokens, num_kv_heads, head_dim]   device, read
+ *   slot_mapping   [num_tokens] int64                      device, read
+ *   key_cache,
+ *   value_cache    [num_blocks, block_size, num_kv_heads, head_dim]  device, written
+ *
+ * For token t with s = slot_mapping[t] >= 0 and every kv head h:
+ *   key_cache[s / block_size, s % block_size, h, :] = key[t, h, :]   (bit copy)
+ * and likewise for V.  s < 0 marks a padding token (skipped).  Slots must be
+ * unique within a call (duplicates race).  A slot >= num_blocks*block_size
+ * is skipped and sets PKV_DEVFLAG_SLOT_RANGE.  num_tokens == 0 is a no-op.
+ */
+pkv_status pkv_kv_cache_write(const void *key, const void *value,
+                              const int64_t *slot_mapping, int64_t num_tokens,
+                              int num_kv_heads, int head_dim,
+                              void *key_cache, void *value_cache,
+                              int64_t num_blocks, int block_size,
+                              pkv_dtype dtype, void *stream);
+
+/*
+ * Partition plan of a decode call: the partition length in tokens the call
+ * will use (a multiple of block_size) and the number of partitions per
+ * sequence (1 = single pass, no workspace).  partition_tokens: > 0 requests
+ * that length (rounded up to a block multiple), 0 = automatic, < 0 = never
+ * split.  Returns PKV_ERR_INVALID_ARG / PKV_ERR_UNSUPPORTED on bad shapes.
+ */
+pkv_status pkv_decode_plan(int batch, int num_heads, int num_kv_heads, int head_dim,
+                           int max_blocks, int block_size, int partition_tokens,
+                           int *plan_partition_tokens, int *plan_num_partitions);
+
+/*
+ * Bytes of device workspace pkv_paged_attention_decode needs for these
+ * arguments (0 when the plan is a single pass).  The workspace holds, per
+ * (sequence, query head, partition), the partition's running max, softmax
+ * normaliser and normalised fp32 output row.
+ */
+size_t pkv_decode_workspace_bytes(int batch, int num_heads, int num_kv_heads, int head_dim,
+                                  int max_blocks, int block_size, int partition_tokens);
+
+/*
+ * paged_attention_decode -- one query token per sequence attends over its
+ * KV cache, scattered across fixed-size physical blocks located through the
+ * block table ([YK] 三 paged_attention_v1; [FC] 二.2 step 3).
+ *
+ *   query          [batch, num_heads, head_dim]                      device, read
+ *   key_cache,
+ *   value_cache    [num_blocks, block_size, num_kv_heads, head_dim]  device, read
+ *   block_tables   [batch, max_blocks] int32                         device, read
+ *   context_lens   [batch] int32                                     device, read
+ *   out            [batch, num_heads, head_dim]                      device, written
+ *   workspace      pkv_decode_workspace_bytes(...) bytes             device, scratch
+ *
+ * For sequence b, query head h (kv head h / (num_heads/num_kv_heads)) and
+ * L = context_lens[b]:
+ *   s_j   = scale * <query[b,h,:], K_j>,   K_j = key_cache[block_tables[b][j / block_size],
+ *                                                          j % block_size, kv_head, :]
+ *   out[b,h,:] = sum_{j<L} softmax(s)_j * V_j          (V_j likewise)
+ * Table entries past ceil(L / block_size) are never read.  L == 0 gives a
+ * zero row.  partition_tokens as for pkv_decode_plan: a split plan computes
+ * each partition's (max, normaliser, output) and merges them by log-sum-exp
+ * in a second kernel.  workspace may be NULL when the plan needs none.
+ */
+pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
+                                      const void *value_cache,
+                                      const int32_t *block_tables, int max_blocks,
+                                      const int32_t *context_lens, int batch,
+                                      int num_heads, int num_kv_heads, int head_dim,
+                                      int block_size, int64_t num_blocks, float scale,
+                                      int partition_tokens, void *workspace,
+                                      size_t workspace_bytes, void *out,
+                                      pkv_dtype dtype, void *stream);
+
+/* ---- host block allocator ([YK] 二; [FC] 二.2 steps 1, 2, 4 and 二.3) ------
+ *
+ * A pool of num_blocks physical block ids with a free list and per-block
+ * reference counts.  It runs on the host only and builds the int32 block
+ * tables the decode call reads.  The free list starts as a permutation of
+ * the ids drawn from `shuffle_seed` (0 = identity order), so a sequence's
+ * blocks are scattered in the pool.  Not thread-safe: one allocator per
+ * thread, or external locking.
+ */
+typedef struct pkv_alloc pkv_alloc;
+
+/* NULL if num_blocks <= 0, block_size <= 0 or host memory is exhausted. */
+pkv_alloc *pkv_alloc_create(int64_t num_blocks, int block_size, uint64_t shuffle_seed);
+void pkv_alloc_destroy(pkv_alloc *a);
+
+int64_t pkv_alloc_num_free(const pkv_alloc *a);
+int pkv_alloc_block_size(const pkv_alloc *a);
+/* Reference count of `block` (0 = free), or -1 if it is outside the pool. */
+int32_t pkv_alloc_refcount(const pkv_alloc *a, int32_t block);
+
+/*
+ * New sequence of num_tokens tokens: takes ceil(num_tokens / block_size)
+ * blocks (refcount 1) into out_blocks[0 .. *n).  PKV_ERR_OOM (nothing taken)
+ * if the pool is short; PKV_ERR_INVALID_ARG if `capacity` is too small.
+ */
+pkv_status pkv_alloc_new_seq(pkv_alloc *a, int64_t num_tokens, int32_t *out_blocks,
+                             int capacity, int *n);
+
+/* Share a sequence's blocks with a forked sequence: refcount + 1 each. */
+pkv_status pkv_alloc_fork(pkv_alloc *a, const int32_t *blocks, int n);
+
+/*
+ * Grow a sequence from old_len to new_len tokens.  blocks[0 .. *n) is its
+ * table (capacity entries).  New blocks are appended as needed.  If old_len
+ * is not a block multiple and the partly filled last block is shared
+ * (refcount > 1), it is first replaced by a fresh block (copy-on-write): the
+ * pair is reported as cow_src[0] -> cow_dst[0] with *n_cow = 1 so the caller
+ * can copy the cells, and the shared block's refcount drops by one.  On
+ * PKV_ERR_OOM nothing changes.
+ */
+pkv_status pkv_alloc_append(pkv_alloc *a, int32_t *blocks, int capacity, int *n,
+                            int64_t old_len, int64_t new_len,
+                            int32_t *cow_src, int32_t *cow_dst, int *n_cow);
+
+/* Release a sequence's blocks: refcount - 1 each; a block reaching 0 returns
+ * to the free list.  PKV_ERR_OUT_OF_RANGE (nothing changed) if an id is
+ * outside the pool or already free. */
+pkv_status pkv_alloc_free(pkv_alloc *a, const int32_t *blocks, int n);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

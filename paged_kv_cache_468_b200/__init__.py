@@ -1,6 +1,21 @@
 """B200-native paged KV-cache decode: the Python face of ``libpagedkv.so``.
 
+    from paged_kv_cache_468_b200 import kv_cache_write, paged_attention_decode
+
 Importing the package loads nothing; the CUDA library is opened on the first
-call that needs it and a missing or unloadable library raises at that point.
+call that needs it, and a missing or unloadable library raises at that point.
 There is no CPU fallback.
 """
+from .pagedkv import (  # noqa: F401
+    BF16,
+    F16,
+    BlockAllocator,
+    PagedKVError,
+    decode_plan,
+    decode_workspace_bytes,
+    device_flags,
+    kv_cache_write,
+    lib,
+    paged_attention_decode,
+    version,
+)

@@ -1,0 +1,390 @@
+// pagedkv.cu -- C-ABI entry points of libpagedkv.so (see include/pagedkv.h).
+//
+// Host-side work only: argument validation, the partition plan, TMA tensor
+// maps, launches.  Every computation of the hot path runs in the kernels of
+// pkv_kernels.cuh.  The library allocates no device memory.
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "pagedkv.h"
+#include "pkv_kernels.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+pkv_status fail(pkv_status s, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+pkv_status fail(pkv_status s, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+pkv_status cuda_fail(cudaError_t e, const char *what)
+{
+    return fail(PKV_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kPlanSmCount = 148;        // B200 SM count used by the automatic plan
+constexpr int kAutoPartitionTokens = 512;
+
+// ---- TMA tensor maps ------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// The cache [num_blocks, bs, Hkv, D] seen as a 3-D tensor
+// (innermost first) {D, Hkv, num_blocks*bs}; a box is 64 columns x 1 head x
+// bs token rows, written to shared memory with the 128-byte swizzle.
+pkv_status make_cache_map(CUtensorMap *map, const void *base, int64_t num_blocks, int bs,
+                          int Hkv, int D, pkv_dtype dt)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)(num_blocks * bs)};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)bs};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = enc(map, dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                     3, const_cast<void *>(base), dims, strides, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return PKV_OK;
+}
+
+// ---- launch configurations ------------------------------------------------
+
+template <int D, int BS>
+struct Tuning;                          // warps per CTA, pipeline depth per warp
+template <> struct Tuning<64, 16>  { static constexpr int NW = 4, S = 4; };
+template <> struct Tuning<64, 32>  { static constexpr int NW = 4, S = 3; };
+template <> struct Tuning<128, 16> { static constexpr int NW = 4, S = 3; };
+template <> struct Tuning<128, 32> { static constexpr int NW = 4, S = 2; };
+
+int current_device()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev;
+}
+
+template <int D, int BS, bool BF16>
+pkv_status launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::DecodeArgs &a,
+                         int batch, int Hkv, cudaStream_t st)
+{
+    constexpr int NW = Tuning<D, BS>::NW;
+    constexpr int S = Tuning<D, BS>::S;
+    using Shape = pkv::DecodeShape<D, BS, NW, S>;
+    auto kern = pkv::paged_decode_kernel<D, BS, BF16, NW, S>;
+    static bool configured[64] = {};
+    static std::mutex mu;
+    const int dev = current_device();
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (dev < 0 || dev >= 64 || !configured[dev]) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 Shape::kSmemBytes);
+            if (e != cudaSuccess)
+                return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+            if (dev >= 0 && dev < 64)
+                configured[dev] = true;
+        }
+    }
+    dim3 grid((unsigned)a.num_parts, (unsigned)Hkv, (unsigned)batch);
+    kern<<<grid, NW * 32, Shape::kSmemBytes, st>>>(mk, mv, a);
+    return PKV_OK;
+}
+
+template <bool BF16>
+pkv_status dispatch_decode(int D, int bs, const CUtensorMap &mk, const CUtensorMap &mv,
+                           const pkv::DecodeArgs &a, int batch, int Hkv, cudaStream_t st)
+{
+    if (D == 64 && bs == 16) return launch_decode<64, 16, BF16>(mk, mv, a, batch, Hkv, st);
+    if (D == 64 && bs == 32) return launch_decode<64, 32, BF16>(mk, mv, a, batch, Hkv, st);
+    if (D == 128 && bs == 16) return launch_decode<128, 16, BF16>(mk, mv, a, batch, Hkv, st);
+    if (D == 128 && bs == 32) return launch_decode<128, 32, BF16>(mk, mv, a, batch, Hkv, st);
+    return fail(PKV_ERR_UNSUPPORTED, "head_dim %d / block_size %d not compiled", D, bs);
+}
+
+pkv_status check_shapes(int batch, int Hq, int Hkv, int D, int max_blocks, int bs)
+{
+    if (batch < 0 || Hq <= 0 || Hkv <= 0 || max_blocks <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "batch=%d num_heads=%d num_kv_heads=%d max_blocks=%d",
+                    batch, Hq, Hkv, max_blocks);
+    if (Hq % Hkv != 0 || Hq / Hkv > 8)
+        return fail(PKV_ERR_UNSUPPORTED, "group size num_heads/num_kv_heads must be an integer 1..8 "
+                    "(num_heads=%d, num_kv_heads=%d)", Hq, Hkv);
+    if (D != 64 && D != 128)
+        return fail(PKV_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", D);
+    if (bs != 16 && bs != 32)
+        return fail(PKV_ERR_UNSUPPORTED, "block_size %d (supported: 16, 32)", bs);
+    if ((int64_t)max_blocks * bs >= (int64_t)1 << 30)
+        return fail(PKV_ERR_INVALID_ARG, "max_blocks * block_size too large");
+    if (batch > 65535 || Hkv > 65535)
+        return fail(PKV_ERR_UNSUPPORTED, "batch and num_kv_heads must be <= 65535");
+    return PKV_OK;
+}
+
+void plan(int batch, int Hkv, int max_blocks, int bs, int requested, int *pt, int *np)
+{
+    const int span = max_blocks * bs;
+    int t = span;
+    if (requested > 0) {
+        t = (requested + bs - 1) / bs * bs;
+    } else if (requested == 0) {
+        const bool long_ctx = span >= 2048;
+        const bool few_items = (int64_t)batch * Hkv < kPlanSmCount;
+        if (long_ctx || few_items)
+            t = kAutoPartitionTokens;
+    }
+    int parts = (span + t - 1) / t;
+    if (parts <= 1) {
+        t = span;
+        parts = 1;
+    }
+    *pt = t;
+    *np = parts;
+}
+
+}  // namespace
+
+// Shared with the allocator's translation unit (not part of the public ABI).
+__attribute__((visibility("hidden"))) void pkv_set_last_error(const char *msg)
+{
+    g_last_error = msg ? msg : "";
+}
+
+extern "C" {
+
+const char *pkv_status_str(pkv_status s)
+{
+    switch (s) {
+    case PKV_OK: return "PKV_OK";
+    case PKV_ERR_INVALID_ARG: return "PKV_ERR_INVALID_ARG";
+    case PKV_ERR_UNSUPPORTED: return "PKV_ERR_UNSUPPORTED";
+    case PKV_ERR_OUT_OF_RANGE: return "PKV_ERR_OUT_OF_RANGE";
+    case PKV_ERR_OOM: return "PKV_ERR_OOM";
+    case PKV_ERR_CUDA: return "PKV_ERR_CUDA";
+    case PKV_ERR_WORKSPACE: return "PKV_ERR_WORKSPACE";
+    case PKV_ERR_MISALIGNED: return "PKV_ERR_MISALIGNED";
+    }
+    return "PKV_ERR_UNKNOWN";
+}
+
+const char *pkv_last_error(void) { return g_last_error.c_str(); }
+
+const char *pkv_version(void) { return "pagedkv 0.1.0 sm_100a"; }
+
+pkv_status pkv_device_flags(int device, unsigned int *flags, int clear)
+{
+    if (!flags)
+        return fail(PKV_ERR_INVALID_ARG, "flags is NULL");
+    int prev = 0;
+    cudaError_t e = cudaGetDevice(&prev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (device != prev && (e = cudaSetDevice(device)) != cudaSuccess)
+        return cuda_fail(e, "cudaSetDevice");
+    pkv_status st = PKV_OK;
+    e = cudaDeviceSynchronize();
+    if (e == cudaSuccess)
+        e = cudaMemcpyFromSymbol(flags, pkv::g_device_flags, sizeof(unsigned int));
+    if (e == cudaSuccess && clear) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(pkv::g_device_flags, &zero, sizeof zero);
+    }
+    if (e != cudaSuccess)
+        st = cuda_fail(e, "reading the device flag word");
+    if (device != prev)
+        cudaSetDevice(prev);
+    return st;
+}
+
+pkv_status pkv_kv_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
+                              int64_t num_tokens, int num_kv_heads, int head_dim, void *key_cache,
+                              void *value_cache, int64_t num_blocks, int block_size,
+                              pkv_dtype dtype, void *stream)
+{
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 || block_size <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_tokens=%lld num_kv_heads=%d head_dim=%d "
+                    "num_blocks=%lld block_size=%d", (long long)num_tokens, num_kv_heads, head_dim,
+                    (long long)num_blocks, block_size);
+    if (dtype != PKV_F16 && dtype != PKV_BF16)
+        return fail(PKV_ERR_INVALID_ARG, "dtype %d", (int)dtype);
+    if ((head_dim * 2) % 16 != 0)
+        return fail(PKV_ERR_UNSUPPORTED, "head_dim %d: rows must be a multiple of 16 bytes", head_dim);
+    if (num_tokens == 0)
+        return PKV_OK;
+    if (!key || !value || !slot_mapping || !key_cache || !value_cache)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(key) || !aligned16(value) || !aligned16(key_cache) || !aligned16(value_cache))
+        return fail(PKV_ERR_MISALIGNED, "key/value/cache pointers must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(slot_mapping) & 7u) != 0)
+        return fail(PKV_ERR_MISALIGNED, "slot_mapping must be 8-byte aligned");
+    const int64_t vec_per_token = (int64_t)num_kv_heads * head_dim / 8;
+    const int64_t n_vec = num_tokens * vec_per_token;
+    const int threads = 256;
+    int64_t blocks = (n_vec + threads - 1) / threads;
+    if (blocks > 148 * 16)
+        blocks = 148 * 16;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    pkv::kv_write_kernel<<<(unsigned)blocks, threads, 0, st>>>(
+        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), slot_mapping, n_vec,
+        vec_per_token, num_blocks * block_size, static_cast<uint4 *>(key_cache),
+        static_cast<uint4 *>(value_cache));
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "kv_write_kernel launch");
+    return PKV_OK;
+}
+
+pkv_status pkv_decode_plan(int batch, int num_heads, int num_kv_heads, int head_dim, int max_blocks,
+                           int block_size, int partition_tokens, int *plan_partition_tokens,
+                           int *plan_num_partitions)
+{
+    pkv_status s = check_shapes(batch, num_heads, num_kv_heads, head_dim, max_blocks, block_size);
+    if (s != PKV_OK)
+        return s;
+    int pt, np;
+    plan(batch, num_kv_heads, max_blocks, block_size, partition_tokens, &pt, &np);
+    if (plan_partition_tokens)
+        *plan_partition_tokens = pt;
+    if (plan_num_partitions)
+        *plan_num_partitions = np;
+    return PKV_OK;
+}
+
+size_t pkv_decode_workspace_bytes(int batch, int num_heads, int num_kv_heads, int head_dim,
+                                  int max_blocks, int block_size, int partition_tokens)
+{
+    if (check_shapes(batch, num_heads, num_kv_heads, head_dim, max_blocks, block_size) != PKV_OK)
+        return 0;
+    int pt, np;
+    plan(batch, num_kv_heads, max_blocks, block_size, partition_tokens, &pt, &np);
+    if (np <= 1)
+        return 0;
+    return (size_t)batch * num_heads * np * (size_t)(head_dim + 2) * sizeof(float);
+}
+
+pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
+                                      const void *value_cache, const int32_t *block_tables,
+                                      int max_blocks, const int32_t *context_lens, int batch,
+                                      int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                      int64_t num_blocks, float scale, int partition_tokens,
+                                      void *workspace, size_t workspace_bytes, void *out,
+                                      pkv_dtype dtype, void *stream)
+{
+    pkv_status s = check_shapes(batch, num_heads, num_kv_heads, head_dim, max_blocks, block_size);
+    if (s != PKV_OK)
+        return s;
+    if (dtype != PKV_F16 && dtype != PKV_BF16)
+        return fail(PKV_ERR_INVALID_ARG, "dtype %d", (int)dtype);
+    if (num_blocks <= 0 || num_blocks * block_size >= ((int64_t)1 << 31))
+        return fail(PKV_ERR_INVALID_ARG, "num_blocks %lld: need 0 < num_blocks*block_size < 2^31",
+                    (long long)num_blocks);
+    if (!std::isfinite(scale))
+        return fail(PKV_ERR_INVALID_ARG, "scale is not finite");
+    if (batch == 0)
+        return PKV_OK;
+    if (!query || !key_cache || !value_cache || !block_tables || !context_lens || !out)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
+        return fail(PKV_ERR_MISALIGNED, "query/cache/out pointers must be 16-byte aligned");
+    if ((reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return fail(PKV_ERR_MISALIGNED, "block_tables/context_lens must be 4-byte aligned");
+
+    int pt, np;
+    plan(batch, num_kv_heads, max_blocks, block_size, partition_tokens, &pt, &np);
+    const size_t need = pkv_decode_workspace_bytes(batch, num_heads, num_kv_heads, head_dim,
+                                                   max_blocks, block_size, partition_tokens);
+    if (np > 1) {
+        if (!workspace || workspace_bytes < need)
+            return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", need,
+                        workspace ? workspace_bytes : (size_t)0);
+        if (!aligned16(workspace))
+            return fail(PKV_ERR_MISALIGNED, "workspace must be 16-byte aligned");
+    }
+
+    CUtensorMap mk, mv;
+    if ((s = make_cache_map(&mk, key_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
+        return s;
+    if ((s = make_cache_map(&mv, value_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
+        return s;
+
+    pkv::DecodeArgs a;
+    a.query = static_cast<const uint16_t *>(query);
+    a.block_tables = block_tables;
+    a.context_lens = context_lens;
+    a.out = static_cast<uint16_t *>(out);
+    const size_t rows = (size_t)batch * num_heads * np;
+    float *ws = static_cast<float *>(workspace);
+    a.ws_m = np > 1 ? ws : nullptr;
+    a.ws_l = np > 1 ? ws + rows : nullptr;
+    a.ws_o = np > 1 ? ws + 2 * rows : nullptr;
+    a.max_blocks = max_blocks;
+    a.num_heads = num_heads;
+    a.group = num_heads / num_kv_heads;
+    a.num_blocks = (int)num_blocks;
+    a.part_tokens = pt;
+    a.num_parts = np;
+    a.scale_log2 = (float)((double)scale * 1.4426950408889634);
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    s = dtype == PKV_BF16 ? dispatch_decode<true>(head_dim, block_size, mk, mv, a, batch, num_kv_heads, st)
+                          : dispatch_decode<false>(head_dim, block_size, mk, mv, a, batch, num_kv_heads, st);
+    if (s != PKV_OK)
+        return s;
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "paged_decode_kernel launch");
+    if (np > 1) {
+        const int span = max_blocks * block_size;
+        if (dtype == PKV_BF16)
+            pkv::lse_merge_kernel<true><<<(unsigned)(batch * num_heads), head_dim, 0, st>>>(
+                a.ws_m, a.ws_l, a.ws_o, context_lens, num_heads, head_dim, np, pt, span, a.out);
+        else
+            pkv::lse_merge_kernel<false><<<(unsigned)(batch * num_heads), head_dim, 0, st>>>(
+                a.ws_m, a.ws_l, a.ws_o, context_lens, num_heads, head_dim, np, pt, span, a.out);
+        e = cudaGetLastError();
+        if (e != cudaSuccess)
+            return cuda_fail(e, "lse_merge_kernel launch");
+    }
+    return PKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,124 @@
+"""The C-ABI library: it builds, loads, exports every declared symbol, and
+validates arguments on the host before touching the GPU (CPU only)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import paged_kv_cache_468_b200 as pkv
+from paged_kv_cache_468_b200 import build, pagedkv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_library_builds():
+    path = build.build()
+    assert os.path.exists(path)
+
+
+def test_every_declared_symbol_is_exported():
+    path = build.build()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = set(re.findall(r"\bT (pkv_[a-z0-9_]+)\b", out))
+    decl = declared_functions()
+    assert len(decl) >= 15
+    missing = [n for n in decl if n not in exported]
+    assert not missing, missing
+    L = pkv.lib()
+    for n in decl:
+        assert hasattr(L, n)
+
+
+def test_status_strings_and_version():
+    assert pagedkv.status_name(0) == "PKV_OK"
+    assert pagedkv.status_name(6) == "PKV_ERR_WORKSPACE"
+    assert "sm_100a" in pkv.version()
+
+
+@pytest.mark.parametrize("args,expect", [
+    ((256, 32, 8, 128, 40, 16, 0), (640, 1)),       # Llama-3-8B-shaped: one pass
+    ((8, 32, 8, 128, 1024, 32, 512), (512, 64)),    # long context: 512-token partitions
+    ((8, 32, 8, 128, 1024, 32, -1), (32768, 1)),    # never split
+    ((8, 32, 8, 128, 1024, 32, 500), (512, 64)),    # rounded up to a block multiple
+    ((4, 8, 8, 64, 13, 16, 0), (208, 1)),           # tiny: one partition covers all
+])
+def test_decode_plan(args, expect):
+    assert pkv.decode_plan(*args) == expect
+
+
+def test_workspace_bytes():
+    # B * Hq * P * (D + 2) floats
+    assert pkv.decode_workspace_bytes(8, 32, 8, 128, 1024, 32, 512) == 8 * 32 * 64 * 130 * 4
+    assert pkv.decode_workspace_bytes(256, 32, 8, 128, 40, 16, 0) == 0
+
+
+@pytest.mark.parametrize("shape,status", [
+    ((4, 8, 3, 64, 4, 16), pagedkv.ERR_UNSUPPORTED),     # 8 % 3 != 0
+    ((4, 32, 2, 64, 4, 16), pagedkv.ERR_UNSUPPORTED),    # group 16 > 8
+    ((4, 8, 8, 96, 4, 16), pagedkv.ERR_UNSUPPORTED),     # head_dim 96
+    ((4, 8, 8, 64, 4, 8), pagedkv.ERR_UNSUPPORTED),      # block_size 8
+    ((4, 8, 8, 64, 0, 16), pagedkv.ERR_INVALID_ARG),     # no table columns
+    ((-1, 8, 8, 64, 4, 16), pagedkv.ERR_INVALID_ARG),
+])
+def test_decode_rejects_shapes_on_host(shape, status):
+    B, Hq, Hkv, D, MB, bs = shape
+    L = pkv.lib()
+    st = L.pkv_paged_attention_decode(None, None, None, None, MB, None, B, Hq, Hkv, D, bs, 100,
+                                      1.0, 0, None, 0, None, 1, None)
+    assert st == status
+    assert L.pkv_last_error()
+
+
+def test_decode_host_validation_before_any_launch():
+    L = pkv.lib()
+    # null pointers
+    assert L.pkv_paged_attention_decode(None, None, None, None, 4, None, 2, 8, 8, 64, 16, 100,
+                                        1.0, 0, None, 0, None, 1, None) == pagedkv.ERR_INVALID_ARG
+    # misaligned (never dereferenced: validation fails first)
+    fake = 0x1008
+    assert L.pkv_paged_attention_decode(fake, fake, fake, fake, 4, fake, 2, 8, 8, 64, 16, 100,
+                                        1.0, 0, None, 0, fake, 1, None) == pagedkv.ERR_MISALIGNED
+    # split plan without workspace
+    a16 = 0x10000
+    assert L.pkv_paged_attention_decode(a16, a16, a16, a16, 1024, a16, 8, 32, 8, 128, 32, 10000,
+                                        1.0, 512, None, 0, a16, 1, None) == pagedkv.ERR_WORKSPACE
+    # non-finite scale, pool too large
+    assert L.pkv_paged_attention_decode(a16, a16, a16, a16, 4, a16, 2, 8, 8, 64, 16, 100,
+                                        float("nan"), 0, None, 0, a16, 1, None) == pagedkv.ERR_INVALID_ARG
+    assert L.pkv_paged_attention_decode(a16, a16, a16, a16, 4, a16, 2, 8, 8, 64, 16, 1 << 28,
+                                        1.0, 0, None, 0, a16, 1, None) == pagedkv.ERR_INVALID_ARG
+    # empty batch is a no-op
+    assert L.pkv_paged_attention_decode(None, None, None, None, 4, None, 0, 8, 8, 64, 16, 100,
+                                        1.0, 0, None, 0, None, 1, None) == pagedkv.OK
+
+
+def test_write_host_validation():
+    L = pkv.lib()
+    assert L.pkv_kv_cache_write(None, None, None, 0, 8, 64, None, None, 10, 16, 1, None) == pagedkv.OK
+    assert L.pkv_kv_cache_write(None, None, None, 3, 8, 64, None, None, 10, 16, 1, None) == pagedkv.ERR_INVALID_ARG
+    f = 0x1004
+    assert L.pkv_kv_cache_write(f, f, f, 3, 8, 64, f, f, 10, 16, 1, None) == pagedkv.ERR_MISALIGNED
+    assert L.pkv_kv_cache_write(None, None, None, -1, 8, 64, None, None, 10, 16, 1, None) == pagedkv.ERR_INVALID_ARG
+    assert L.pkv_kv_cache_write(None, None, None, 1, 8, 64, None, None, 10, 16, 7, None) == pagedkv.ERR_INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    q = torch.zeros(2, 8, 64, dtype=torch.float16)
+    kc = torch.zeros(4, 16, 8, 64, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        pkv.paged_attention_decode(q, kc, kc.clone(), torch.zeros(2, 4, dtype=torch.int32),
+                                   torch.ones(2, dtype=torch.int32), 0.125)
