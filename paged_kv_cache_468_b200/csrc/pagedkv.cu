@@ -89,12 +89,21 @@ pkv_status make_cache_map(CUtensorMap *map, const void *base, int64_t num_blocks
 
 // ---- launch configurations ------------------------------------------------
 
+// Warps per CTA and pipeline depth (stages per warp), chosen by sweeping on
+// B200: several small CTAs per SM hide each CTA's start-up (table lookup ->
+// TMA -> first data) behind the others' streaming.  PKV_TUNE_NW / PKV_TUNE_S
+// override every shape at build time (used for tuning sweeps).
 template <int D, int BS>
-struct Tuning;                          // warps per CTA, pipeline depth per warp
-template <> struct Tuning<64, 16>  { static constexpr int NW = 4, S = 4; };
-template <> struct Tuning<64, 32>  { static constexpr int NW = 4, S = 3; };
-template <> struct Tuning<128, 16> { static constexpr int NW = 4, S = 3; };
-template <> struct Tuning<128, 32> { static constexpr int NW = 4, S = 2; };
+struct Tuning;
+#if defined(PKV_TUNE_NW) && defined(PKV_TUNE_S)
+template <int D, int BS>
+struct Tuning { static constexpr int NW = PKV_TUNE_NW, S = PKV_TUNE_S; };
+#else
+template <> struct Tuning<64, 16>  { static constexpr int NW = 4, S = 2; };   // 33 KB, 6 CTAs/SM
+template <> struct Tuning<64, 32>  { static constexpr int NW = 2, S = 3; };   // 49 KB
+template <> struct Tuning<128, 16> { static constexpr int NW = 4, S = 2; };   // 65 KB, 3 CTAs/SM
+template <> struct Tuning<128, 32> { static constexpr int NW = 2, S = 3; };   // 97 KB, 2 CTAs/SM
+#endif
 
 int current_device()
 {
