@@ -161,6 +161,32 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
                                       size_t workspace_bytes, void *out,
                                       pkv_dtype dtype, void *stream);
 
+/*
+ * paged_attention_decode_static_workspace -- the same decode as
+ * pkv_paged_attention_decode, for callers that cannot allocate device memory
+ * at call time (an allocator that owns the whole pool, a serving runtime that
+ * forbids cudaMalloc on its hot path, C code without an allocator).  The
+ * pages have no counterpart: this is a convenience of this library.
+ *
+ * Arguments are those of pkv_paged_attention_decode without the workspace.
+ * A split plan's workspace is taken from an array of
+ * PKV_STATIC_WORKSPACE_BYTES bytes that the library reserves in device memory
+ * on every GPU that loads it, until the process exits; nothing is allocated
+ * per call.  The first call on a device looks up that array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array, which keeps the
+ * last call's contents (no part of it needs to start at zero): calls whose
+ * kernels overlap on the GPU race and must be serialised by the caller.  A
+ * plan needing more than PKV_STATIC_WORKSPACE_BYTES returns
+ * PKV_ERR_WORKSPACE without launching anything.
+ */
+#define PKV_STATIC_WORKSPACE_BYTES (16u << 20)   /* 16 MiB per device */
+pkv_status pkv_paged_attention_decode_static_workspace(
+    const void *query, const void *key_cache, const void *value_cache,
+    const int32_t *block_tables, int max_blocks, const int32_t *context_lens, int batch,
+    int num_heads, int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+    float scale, int partition_tokens, void *out, pkv_dtype dtype, void *stream);
+
 /* ---- host block allocator ([YK] 二; [FC] 二.2 steps 1, 2, 4 and 二.3) ------
  *
  * A pool of num_blocks physical block ids with a free list and per-block

@@ -397,3 +397,77 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode with a library-owned workspace (no allocation by anyone at call time)
+// ---------------------------------------------------------------------------
+// Some callers cannot allocate device memory when they decode: a custom
+// allocator that owns the whole pool, a runtime that forbids cudaMalloc on its
+// serving path, or plain C code with no allocator at all.  For them the split
+// plan's workspace lives in this fixed array, reserved in device memory on
+// every GPU that loads the library and kept until the process exits.  Calls
+// share it, so two calls whose kernels overlap on the GPU (different streams,
+// or different host threads) race on it and must be serialised by the caller.
+// The array keeps whatever the last call left; nothing in it has to start at
+// zero, because every partition record the merge reads is written earlier in
+// the same call.
+namespace {
+
+constexpr size_t kStaticWorkspaceBytes = PKV_STATIC_WORKSPACE_BYTES;
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+// Device address of g_static_workspace on `dev`, looked up once per device
+// with that device current.  In host code the symbol is only a stand-in for
+// the device array, so its address must come from cudaGetSymbolAddress.
+pkv_status static_workspace_ptr(int dev, void **ptr)
+{
+    static void *cache[64] = {};
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < 64 && cache[dev]) {
+        *ptr = cache[dev];
+        return PKV_OK;
+    }
+    void *p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
+    if (dev >= 0 && dev < 64)
+        cache[dev] = p;
+    *ptr = p;
+    return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" pkv_status pkv_paged_attention_decode_static_workspace(
+    const void *query, const void *key_cache, const void *value_cache, const int32_t *block_tables,
+    int max_blocks, const int32_t *context_lens, int batch, int num_heads, int num_kv_heads,
+    int head_dim, int block_size, int64_t num_blocks, float scale, int partition_tokens, void *out,
+    pkv_dtype dtype, void *stream)
+{
+    pkv_status s = check_shapes(batch, num_heads, num_kv_heads, head_dim, max_blocks, block_size);
+    if (s != PKV_OK)
+        return s;
+    const size_t need = pkv_decode_workspace_bytes(batch, num_heads, num_kv_heads, head_dim,
+                                                   max_blocks, block_size, partition_tokens);
+    if (need > kStaticWorkspaceBytes)
+        return fail(PKV_ERR_WORKSPACE,
+                    "this call needs %zu bytes of workspace but the library's static workspace "
+                    "holds %zu (PKV_STATIC_WORKSPACE_BYTES); use pkv_paged_attention_decode with a "
+                    "caller-provided workspace, fewer partitions or a smaller batch",
+                    need, kStaticWorkspaceBytes);
+    void *ws = nullptr;
+    if (need > 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetDevice");
+        if ((s = static_workspace_ptr(dev, &ws)) != PKV_OK)
+            return s;
+    }
+    return pkv_paged_attention_decode(query, key_cache, value_cache, block_tables, max_blocks,
+                                      context_lens, batch, num_heads, num_kv_heads, head_dim,
+                                      block_size, num_blocks, scale, partition_tokens, ws,
+                                      need > 0 ? kStaticWorkspaceBytes : 0, out, dtype, stream);
+}
