@@ -323,10 +323,8 @@ def run_gpu(args, cfg, world, rank, local):
         one_step()
     torch.cuda.synchronize()
 
-    # ---- device-timed region (inputs resident in HBM) ----
+    # ---- device-timed region (inputs resident in HBM): K whole steps ----
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(K)]
     sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
     if sampler:
         sampler.start()
@@ -337,14 +335,8 @@ def run_gpu(args, cfg, world, rank, local):
     if sampler:
         sampler.mark(True)
     t_start.record(stream)
-    for i in range(K):
-        pkv.kv_cache_write(d["new_key"], d["new_value"], d["slot_mapping"], d["key_cache"],
-                           d["value_cache"])
-        ev[i][0].record(stream)
-        pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
-                                   d["context_lens"], d["scale"], partition_tokens=pt_req,
-                                   out=out, workspace=ws)
-        ev[i][1].record(stream)
+    for _ in range(K):
+        one_step()
     t_end.record(stream)
     torch.cuda.synchronize()
     if sampler:
@@ -352,8 +344,22 @@ def run_gpu(args, cfg, world, rank, local):
     barrier(world)
     ms_total = t_start.elapsed_time(t_end)
     ms_total_max = max_over_ranks(ms_total, world)
-    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)   # decode (+ merge) per launch
     clocks = sampler.stop() if sampler else None
+
+    # ---- the decode call alone (its kernels), for the roofline: CUDA events
+    # around each launch on the launching stream ----
+    Kd = max(1, min(K, args.roofline_launches))
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(Kd)]
+    torch.cuda.synchronize()
+    for i in range(Kd):
+        ev[i][0].record(stream)
+        pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
+                                   d["context_lens"], d["scale"], partition_tokens=pt_req,
+                                   out=out, workspace=ws)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)   # decode (+ merge) per call
     flags = pkv.device_flags(clear=True)
 
     # ---- end to end through the public API, host buffers ----
@@ -441,6 +447,7 @@ def run_gpu(args, cfg, world, rank, local):
             "frac_of_hbm_peak": round(value / peaks["hbm_gbs"], 4),
             "logical_kv_gbs": round(sum_over_ranks(nbytes["kv"], world) / (ms_step * 1e-3) / 1e9, 1),
             "gpu_launches": launches_per_step * K,
+            "launches_per_step": launches_per_step,
             "device_flags": flags,
             "roofline": roofline,
             "clocks": clocks,
@@ -466,6 +473,7 @@ def main(argv=None):
     ap.add_argument("--partition-tokens", type=int, default=None,
                     help="override the workload's partition request (0 auto, <0 never)")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--roofline-launches", type=int, default=500)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--no-e2e", action="store_true")

@@ -112,6 +112,26 @@ int current_device()
     return dev;
 }
 
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel on the stream finishes; it waits (griddepcontrol.wait)
+// before it reads any memory.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 template <int D, int BS, bool BF16>
 pkv_status launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::DecodeArgs &a,
                          int batch, int Hkv, cudaStream_t st)
@@ -135,7 +155,9 @@ pkv_status launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pkv
         }
     }
     dim3 grid((unsigned)a.num_parts, (unsigned)Hkv, (unsigned)batch);
-    kern<<<grid, NW * 32, Shape::kSmemBytes, st>>>(mk, mv, a);
+    cudaError_t e = launch_pdl(kern, grid, dim3(NW * 32), Shape::kSmemBytes, st, mk, mv, a);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "paged_decode_kernel launch");
     return PKV_OK;
 }
 
@@ -383,13 +405,20 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
         return cuda_fail(e, "paged_decode_kernel launch");
     if (np > 1) {
         const int span = max_blocks * block_size;
+        constexpr int NT = 512;
+        const dim3 mgrid((unsigned)((size_t)batch * num_heads));
         if (dtype == PKV_BF16)
-            pkv::lse_merge_kernel<true><<<(unsigned)(batch * num_heads), head_dim, 0, st>>>(
-                a.ws_m, a.ws_l, a.ws_o, context_lens, num_heads, head_dim, np, pt, span, a.out);
+            e = head_dim == 64
+                    ? launch_pdl(pkv::lse_merge_kernel<true, 64, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
+                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out)
+                    : launch_pdl(pkv::lse_merge_kernel<true, 128, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
+                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out);
         else
-            pkv::lse_merge_kernel<false><<<(unsigned)(batch * num_heads), head_dim, 0, st>>>(
-                a.ws_m, a.ws_l, a.ws_o, context_lens, num_heads, head_dim, np, pt, span, a.out);
-        e = cudaGetLastError();
+            e = head_dim == 64
+                    ? launch_pdl(pkv::lse_merge_kernel<false, 64, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
+                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out)
+                    : launch_pdl(pkv::lse_merge_kernel<false, 128, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
+                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out);
         if (e != cudaSuccess)
             return cuda_fail(e, "lse_merge_kernel launch");
     }

@@ -98,6 +98,9 @@ __global__ void kv_write_kernel(const uint4 *__restrict__ key, const uint4 *__re
                                 int64_t vec_per_token, int64_t total_slots,
                                 uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache)
 {
+    // A decode launched after this kernel may start its own set-up now; it
+    // waits for this grid to finish before it reads any memory.
+    asm volatile("griddepcontrol.launch_dependents;");
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += stride) {
         const int64_t t = i / vec_per_token;
@@ -177,7 +180,51 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int G = a.group;
     const bool split = a.num_parts > 1;
 
+    // Set-up that touches no global memory, then wait for the previous kernel
+    // on the stream (programmatic dependent launch lets this CTA start while
+    // it finishes; it may have written the caches or this call's inputs).
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < S; ++s)
+            mbar_init(smem_addr(&bars[warp * S + s]), 1);
+    }
+    if (threadIdx.x == 0) {
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    fence_mbar_init();
+    __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    // The context length, this warp's first 32 table entries and the query are
+    // loaded together: the table window is bounded by the partition and the
+    // row, not by the length, so it does not wait for it.
+    const int blk0 = (part * a.part_tokens) / BS;
+    const int part_blocks = a.part_tokens / BS;
+    const int32_t *trow = a.block_tables + (size_t)b * a.max_blocks + blk0 + warp;
+    int ids;   // lane j holds the physical id of this warp's block (window*32 + j)
+    {
+        const int lb = warp + lane * NW;   // block of window 0 within the partition
+        ids = (lb < part_blocks && blk0 + lb < a.max_blocks) ? __ldg(trow + (size_t)lane * NW) : 0;
+    }
     int L = __ldg(a.context_lens + b);
+
+    // Q^T as the B operand of S^T = K Q^T: column n = query head kvh*G + n of
+    // the group (n >= G are zero columns), row k = head-dim index.
+    uint32_t qf[KS][2];
+    {
+        const int n = lane >> 2;
+        const int c = lane & 3;
+        const uint32_t *q32 = reinterpret_cast<const uint32_t *>(
+            a.query + ((size_t)b * Hq + (size_t)kvh * G + (n < G ? n : 0)) * D);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qf[ks][0] = n < G ? __ldg(q32 + ks * 8 + c) : 0u;
+            qf[ks][1] = n < G ? __ldg(q32 + ks * 8 + 4 + c) : 0u;
+        }
+    }
+
     const int span = a.max_blocks * BS;
     if (L < 0 || L > span) {
         if (threadIdx.x == 0 && part == 0 && kvh == 0)
@@ -198,46 +245,16 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         return;
     }
     const int nblk = (tok1 - tok0 + BS - 1) / BS;
-    const int blk0 = tok0 / BS;
-
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < S; ++s)
-            mbar_init(smem_addr(&bars[warp * S + s]), 1);
-    }
-    if (threadIdx.x == 0) {
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-    }
-    fence_mbar_init();
-    __syncthreads();
-
-    // Q^T as the B operand of S^T = K Q^T: column n = query head kvh*G + n of
-    // the group (n >= G are zero columns), row k = head-dim index.
-    uint32_t qf[KS][2];
-    {
-        const int n = lane >> 2;
-        const int c = lane & 3;
-        const uint32_t *q32 = reinterpret_cast<const uint32_t *>(
-            a.query + ((size_t)b * Hq + (size_t)kvh * G + (n < G ? n : 0)) * D);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qf[ks][0] = n < G ? __ldg(q32 + ks * 8 + c) : 0u;
-            qf[ks][1] = n < G ? __ldg(q32 + ks * 8 + 4 + c) : 0u;
-        }
-    }
 
     // This warp's blocks: logical blocks blk0 + warp + k*NW, k = 0 .. nk-1.
     const int nk = nblk > warp ? (nblk - warp + NW - 1) / NW : 0;
-    const int32_t *trow = a.block_tables + (size_t)b * a.max_blocks + blk0 + warp;
     uint8_t *ring = smem + (size_t)warp * S * kStageBytes;
     const uint32_t ring_s = smem_addr(ring);
     const uint32_t bar0 = smem_addr(&bars[warp * S]);
     const uint64_t policy = policy_evict_first();
 
-    int ids = 0;   // lane j holds the physical id of this warp's block (window*32 + j)
     auto issue = [&](int k) {
-        if ((k & 31) == 0) {
+        if ((k & 31) == 0 && k > 0) {
             const int kk = k + lane;
             ids = kk < nk ? __ldg(trow + (size_t)kk * NW) : 0;
         }
@@ -314,9 +331,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         float sc[MT][4];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                sc[mt][i] = 0.f;
+            float s0[4] = {0.f, 0.f, 0.f, 0.f};   // two accumulation chains (even / odd k)
+            float s1[4] = {0.f, 0.f, 0.f, 0.f};
             const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
             for (int ks = 0; ks < KS; ++ks) {
@@ -325,8 +341,14 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                                                       ((chunk ^ (row & 7)) << 4));
                 uint32_t af[4];
                 ldsm_x4(addr, af);
-                mma_16816<BF16>(sc[mt], af, qf[ks][0], qf[ks][1]);
+                if (ks & 1)
+                    mma_16816<BF16>(s1, af, qf[ks][0], qf[ks][1]);
+                else
+                    mma_16816<BF16>(s0, af, qf[ks][0], qf[ks][1]);
             }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                sc[mt][i] = s0[i] + s1[i];
         }
 
         // ---- online softmax (base 2), per column n = 2c + j ----
@@ -480,32 +502,64 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // ---------------------------------------------------------------------------
 // Log-sum-exp merge of split partitions
 // ---------------------------------------------------------------------------
-// One CTA per (sequence, query head) row.  out = sum_p w_p o_p / sum_p w_p with
-// w_p = 2^(m_p - M) l_p, M = max_p m_p, over the partitions that hold tokens.
-template <bool BF16>
-__global__ void lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
-                                 const float *__restrict__ ws_o,
-                                 const int32_t *__restrict__ context_lens, int num_heads, int D,
-                                 int num_parts, int part_tokens, int span, uint16_t *__restrict__ out)
+// One CTA per (sequence, query head) row; NT threads = NG groups of D, group q
+// folds partitions q, q + NG, ... with an online log-sum-exp, then the groups
+// are combined.  out = sum_p w_p o_p / sum_p w_p with w_p = 2^(m_p - M) l_p,
+// M = max_p m_p, over the partitions that hold tokens.  Launched with
+// programmatic dependent launch: it waits for the decode kernel first.
+template <bool BF16, int D, int NT>
+__global__ void __launch_bounds__(NT)
+lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
+                 const float *__restrict__ ws_o, const int32_t *__restrict__ context_lens,
+                 int num_heads, int num_parts, int part_tokens, int span, uint16_t *__restrict__ out)
 {
+    constexpr int NG = NT / D;
+    __shared__ float s_M[NG][D], s_den[NG][D], s_num[NG][D];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     const size_t row = blockIdx.x;
+    const int d = threadIdx.x % D;
+    const int grp = threadIdx.x / D;
     const int b = (int)(row / num_heads);
     int L = __ldg(context_lens + b);
     L = L < 0 ? 0 : (L > span ? span : L);
     const int np = (L + part_tokens - 1) / part_tokens;
     const float *m = ws_m + row * num_parts;
     const float *l = ws_l + row * num_parts;
-    float M = kNegInf;
-    for (int p = 0; p < np; ++p)
-        M = fmaxf(M, __ldg(m + p));
-    for (int d = threadIdx.x; d < D; d += blockDim.x) {
-        float den = 0.f, num = 0.f;
-        for (int p = 0; p < np; ++p) {
-            const float w = ex2(__ldg(m + p) - M) * __ldg(l + p);
-            den += w;
-            num += w * __ldg(ws_o + (row * num_parts + p) * D + d);
+    const float *o = ws_o + row * num_parts * D + d;
+    float M = kNegInf, den = 0.f, num = 0.f;
+#pragma unroll 4
+    for (int p = grp; p < np; p += NG) {
+        const float mp = __ldg(m + p);
+        const float lp = __ldg(l + p);
+        const float op = __ldg(o + (size_t)p * D);
+        if (mp > M) {
+            const float sc = ex2(M - mp);   // 0 while M is -inf
+            den *= sc;
+            num *= sc;
+            M = mp;
         }
-        out[row * D + d] = to_storage<BF16>(den > 0.f ? num / den : 0.f);
+        const float w = ex2(mp - M) * lp;
+        den += w;
+        num += w * op;
+    }
+    s_M[grp][d] = M;
+    s_den[grp][d] = den;
+    s_num[grp][d] = num;
+    __syncthreads();
+    if (grp == 0) {
+        float Mt = kNegInf;
+#pragma unroll
+        for (int q = 0; q < NG; ++q)
+            Mt = fmaxf(Mt, s_M[q][d]);
+        float dt = 0.f, nt = 0.f;
+#pragma unroll
+        for (int q = 0; q < NG; ++q) {
+            const float e = ex2(s_M[q][d] - Mt);   // 0 for groups that held no partition
+            dt += e * s_den[q][d];
+            nt += e * s_num[q][d];
+        }
+        out[row * D + d] = to_storage<BF16>(dt > 0.f ? nt / dt : 0.f);
     }
 }
 
