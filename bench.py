@@ -197,22 +197,36 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Job time = the slowest rank's (all ranks take part)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def sum_over_ranks(x: float, world: int) -> float:
+def sum_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """Work of the whole job = the sum of every rank's (all ranks take part)."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
+
+
+def replica_seed(cfg_seed: int, rank: int) -> int:
+    """Each rank draws its own replica of the workload (its own sequences)."""
+    return cfg_seed + 1000 * rank
+
+
+def job_throughput(bytes_local: float, ms_local: float, world: int, device: str = "cuda") -> tuple:
+    """(GB/s of the whole job, job ms): all ranks' bytes over the slowest rank's time."""
+    ms = max_over_ranks(ms_local, world, device)
+    total = sum_over_ranks(bytes_local, world, device)
+    return total / (ms * 1e-3) / 1e9, ms
 
 
 # ------------------------------------------------------- CPU oracle timing --
@@ -297,7 +311,7 @@ def run_gpu(args, cfg, world, rank, local):
     import paged_kv_cache_468_b200 as pkv
 
     dev = torch.device("cuda", local)
-    step = workloads.make_decode_step(dataclass_replace(cfg, seed=cfg.seed + 1000 * rank))
+    step = workloads.make_decode_step(dataclass_replace(cfg, seed=replica_seed(cfg.seed, rank)))
     nbytes = step_bytes(step, cfg)
     d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
     B, Hq, D = d["query"].shape
@@ -343,7 +357,6 @@ def run_gpu(args, cfg, world, rank, local):
         sampler.mark(False)
     barrier(world)
     ms_total = t_start.elapsed_time(t_end)
-    ms_total_max = max_over_ranks(ms_total, world)
     clocks = sampler.stop() if sampler else None
 
     # ---- the decode call alone (its kernels), for the roofline: CUDA events
@@ -402,10 +415,11 @@ def run_gpu(args, cfg, world, rank, local):
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": Ke,
                "tokens_per_s": round(sum_over_ranks(B, world) / (e2e_ms * 1e-3), 1)}
 
-    ms_step = ms_total_max / K
-    total_bytes = sum_over_ranks(nbytes["decode"] + nbytes["write"], world)
-    value = total_bytes / (ms_step * 1e-3) / 1e9
+    value, ms_step = job_throughput(nbytes["decode"] + nbytes["write"], ms_total / K, world)
+    # every collective before any rank-0-only code: all ranks take the same steps
     tokens = sum_over_ranks(B, world)
+    kv_tokens_all = sum_over_ranks(nbytes["kv_tokens"], world)
+    kv_all = sum_over_ranks(nbytes["kv"], world)
 
     peaks = measured_peaks()
     achieved = nbytes["decode_unique"] / (decode_ms * 1e-3) / 1e9
@@ -443,9 +457,9 @@ def run_gpu(args, cfg, world, rank, local):
                               f"per step vs 126 MB L2, no flush")
                        if nbytes["kv_unique"] > 126e6 else "inputs fit in L2 (no flush)"},
             "tokens_per_s": round(tokens / (ms_step * 1e-3), 1),
-            "kv_tokens_per_s": round(sum_over_ranks(nbytes["kv_tokens"], world) / (ms_step * 1e-3), 1),
+            "kv_tokens_per_s": round(kv_tokens_all / (ms_step * 1e-3), 1),
             "frac_of_hbm_peak": round(value / peaks["hbm_gbs"], 4),
-            "logical_kv_gbs": round(sum_over_ranks(nbytes["kv"], world) / (ms_step * 1e-3) / 1e9, 1),
+            "logical_kv_gbs": round(kv_all / (ms_step * 1e-3) / 1e9, 1),
             "gpu_launches": launches_per_step * K,
             "launches_per_step": launches_per_step,
             "device_flags": flags,

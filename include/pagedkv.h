@@ -87,6 +87,15 @@ const char *pkv_version(void);
 pkv_status pkv_device_flags(int device, unsigned int *flags, int clear);
 
 /*
+ * Failure-detection self-test: launches one warp that waits, through the
+ * decode kernel's bounded shared-memory pipeline wait, on a barrier phase
+ * that nothing completes.  After limit_ns (0 < limit_ns <= 1e10) the wait
+ * gives up, PKV_DEVFLAG_WAIT_TIMEOUT is set and the kernel returns; the
+ * context stays usable.  Asynchronous on `stream`.
+ */
+pkv_status pkv_selftest_bounded_wait(int64_t limit_ns, void *stream);
+
+/*
  * kv_cache_write -- store the current tokens' K/V into their cache cells
  * ([MH] 2.1, 3.3; cache shape [YK] 三).
  *

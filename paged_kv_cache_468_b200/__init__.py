@@ -17,5 +17,6 @@ from .pagedkv import (  # noqa: F401
     kv_cache_write,
     lib,
     paged_attention_decode,
+    selftest_bounded_wait,
     version,
 )

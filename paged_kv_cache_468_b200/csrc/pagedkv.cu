@@ -132,6 +132,30 @@ cudaError_t launch_pdl(Kernel kern, dim3 grid, dim3 block, size_t smem, cudaStre
     return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
+// Merge launch: 512 threads per CTA; with at most 8 partitions per row each
+// 128/64-thread group merges its own row, otherwise the groups split a row.
+template <bool BF16, int D>
+cudaError_t launch_merge_d(const pkv::DecodeArgs &a, const int32_t *context_lens, int rows,
+                           int Hq, int np, int pt, int span, cudaStream_t st)
+{
+    constexpr int NT = 512, NG = NT / D;
+    if (np <= 8)
+        return launch_pdl(pkv::lse_merge_kernel<BF16, D, NT, NG>, dim3((unsigned)((rows + NG - 1) / NG)),
+                          dim3(NT), 0, st, a.ws_m, a.ws_l, a.ws_o, context_lens, Hq, rows, np, pt,
+                          span, a.out);
+    return launch_pdl(pkv::lse_merge_kernel<BF16, D, NT, 1>, dim3((unsigned)rows), dim3(NT), 0, st,
+                      a.ws_m, a.ws_l, a.ws_o, context_lens, Hq, rows, np, pt, span, a.out);
+}
+
+template <bool BF16>
+cudaError_t launch_merge(int D, const pkv::DecodeArgs &a, const int32_t *context_lens, int batch,
+                         int Hq, int np, int pt, int span, cudaStream_t st)
+{
+    const int rows = batch * Hq;
+    return D == 64 ? launch_merge_d<BF16, 64>(a, context_lens, rows, Hq, np, pt, span, st)
+                   : launch_merge_d<BF16, 128>(a, context_lens, rows, Hq, np, pt, span, st);
+}
+
 template <int D, int BS, bool BF16>
 pkv_status launch_decode(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::DecodeArgs &a,
                          int batch, int Hkv, cudaStream_t st)
@@ -264,6 +288,18 @@ pkv_status pkv_device_flags(int device, unsigned int *flags, int clear)
     if (device != prev)
         cudaSetDevice(prev);
     return st;
+}
+
+pkv_status pkv_selftest_bounded_wait(int64_t limit_ns, void *stream)
+{
+    if (limit_ns <= 0 || limit_ns > 10000000000ll)
+        return fail(PKV_ERR_INVALID_ARG, "limit_ns must be in (0, 1e10]");
+    pkv::bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        (uint64_t)limit_ns);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "bounded_wait_selftest_kernel launch");
+    return PKV_OK;
 }
 
 pkv_status pkv_kv_cache_write(const void *key, const void *value, const int64_t *slot_mapping,
@@ -404,21 +440,10 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
     if (e != cudaSuccess)
         return cuda_fail(e, "paged_decode_kernel launch");
     if (np > 1) {
-        const int span = max_blocks * block_size;
-        constexpr int NT = 512;
-        const dim3 mgrid((unsigned)((size_t)batch * num_heads));
-        if (dtype == PKV_BF16)
-            e = head_dim == 64
-                    ? launch_pdl(pkv::lse_merge_kernel<true, 64, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
-                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out)
-                    : launch_pdl(pkv::lse_merge_kernel<true, 128, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
-                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out);
-        else
-            e = head_dim == 64
-                    ? launch_pdl(pkv::lse_merge_kernel<false, 64, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
-                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out)
-                    : launch_pdl(pkv::lse_merge_kernel<false, 128, NT>, mgrid, dim3(NT), 0, st, a.ws_m,
-                                 a.ws_l, a.ws_o, context_lens, num_heads, np, pt, span, a.out);
+        e = dtype == PKV_BF16 ? launch_merge<true>(head_dim, a, context_lens, batch, num_heads, np, pt,
+                                                   max_blocks * block_size, st)
+                              : launch_merge<false>(head_dim, a, context_lens, batch, num_heads, np,
+                                                    pt, max_blocks * block_size, st);
         if (e != cudaSuccess)
             return cuda_fail(e, "lse_merge_kernel launch");
     }

@@ -500,26 +500,50 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 }
 
 // ---------------------------------------------------------------------------
+// Self-test of the bounded pipeline wait
+// ---------------------------------------------------------------------------
+// One warp waits, through the same bounded wait the decode kernel uses, on an
+// mbarrier phase that nothing completes; after limit_ns it must give up, set
+// PKV_DEVFLAG_WAIT_TIMEOUT and return, leaving the context usable.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns)
+{
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0)
+        mbar_init(smem_addr(&bar), 1);
+    fence_mbar_init();
+    __syncwarp();
+    const bool got = mbar_wait_bounded(smem_addr(&bar), 0u, limit_ns);
+    if (!__all_sync(0xffffffffu, got) && threadIdx.x == 0)
+        raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
 // Log-sum-exp merge of split partitions
 // ---------------------------------------------------------------------------
-// One CTA per (sequence, query head) row; NT threads = NG groups of D, group q
-// folds partitions q, q + NG, ... with an online log-sum-exp, then the groups
-// are combined.  out = sum_p w_p o_p / sum_p w_p with w_p = 2^(m_p - M) l_p,
-// M = max_p m_p, over the partitions that hold tokens.  Launched with
-// programmatic dependent launch: it waits for the decode kernel first.
-template <bool BF16, int D, int NT>
+// One CTA per RPC (sequence, query head) rows.  NT threads = NG groups of D.  With RPC == NG each group merges its own
+// (sequence, query head) row over all of its partitions (plans with few
+// partitions: fewer, fuller CTAs); with RPC == 1 the groups fold one row's
+// partitions q, q + NG, ... with an online log-sum-exp and are then combined
+// (plans with many partitions).  out = sum_p w_p o_p / sum_p w_p,
+// w_p = 2^(m_p - M) l_p, M = max_p m_p, over the partitions that hold tokens.
+// Launched with programmatic dependent launch: it waits for the decode first.
+template <bool BF16, int D, int NT, int RPC>
 __global__ void __launch_bounds__(NT)
 lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
                  const float *__restrict__ ws_o, const int32_t *__restrict__ context_lens,
-                 int num_heads, int num_parts, int part_tokens, int span, uint16_t *__restrict__ out)
+                 int num_heads, int num_rows, int num_parts, int part_tokens, int span,
+                 uint16_t *__restrict__ out)
 {
     constexpr int NG = NT / D;
+    static_assert(RPC == 1 || RPC == NG, "rows per CTA");
     __shared__ float s_M[NG][D], s_den[NG][D], s_num[NG][D];
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    const size_t row = blockIdx.x;
     const int d = threadIdx.x % D;
     const int grp = threadIdx.x / D;
+    const size_t row = (size_t)blockIdx.x * RPC + (RPC == 1 ? 0 : grp);
+    if (row >= (size_t)num_rows)
+        return;                                  // (RPC > 1: no barrier follows)
     const int b = (int)(row / num_heads);
     int L = __ldg(context_lens + b);
     L = L < 0 ? 0 : (L > span ? span : L);
@@ -527,9 +551,11 @@ lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
     const float *m = ws_m + row * num_parts;
     const float *l = ws_l + row * num_parts;
     const float *o = ws_o + row * num_parts * D + d;
+    const int p0 = RPC == 1 ? grp : 0;
+    const int pstep = RPC == 1 ? NG : 1;
     float M = kNegInf, den = 0.f, num = 0.f;
 #pragma unroll 4
-    for (int p = grp; p < np; p += NG) {
+    for (int p = p0; p < np; p += pstep) {
         const float mp = __ldg(m + p);
         const float lp = __ldg(l + p);
         const float op = __ldg(o + (size_t)p * D);
@@ -542,6 +568,10 @@ lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
         const float w = ex2(mp - M) * lp;
         den += w;
         num += w * op;
+    }
+    if (RPC > 1) {
+        out[row * D + d] = to_storage<BF16>(den > 0.f ? num / den : 0.f);
+        return;
     }
     s_M[grp][d] = M;
     s_den[grp][d] = den;

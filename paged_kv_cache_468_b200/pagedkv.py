@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_version.argtypes = []
         L.pkv_device_flags.restype = i32
         L.pkv_device_flags.argtypes = [i32, ctypes.POINTER(ctypes.c_uint), i32]
+        L.pkv_selftest_bounded_wait.restype = i32
+        L.pkv_selftest_bounded_wait.argtypes = [i64, P]
         L.pkv_kv_cache_write.restype = i32
         L.pkv_kv_cache_write.argtypes = [P, P, P, i64, i32, i32, P, P, i64, i32, i32, P]
         L.pkv_decode_plan.restype = i32
@@ -125,6 +127,13 @@ def device_flags(device: Optional[int] = None, clear: bool = True) -> int:
     v = ctypes.c_uint(0)
     _check(lib().pkv_device_flags(dev, ctypes.byref(v), int(clear)), "pkv_device_flags")
     return v.value
+
+
+def selftest_bounded_wait(limit_ns: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Launch the bounded-wait self-test kernel (see pkv_selftest_bounded_wait)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib().pkv_selftest_bounded_wait(int(limit_ns), _stream_handle(stream, dev)),
+           "pkv_selftest_bounded_wait")
 
 
 def kv_cache_write(key: torch.Tensor, value: torch.Tensor, slot_mapping: torch.Tensor,
