@@ -320,17 +320,34 @@ def run_gpu(args, cfg, world, rank, local):
     pt_req = cfg.partition_tokens if args.partition_tokens is None else args.partition_tokens
     plan_pt, plan_np = pkv.decode_plan(B, Hq, Hkv, D, MB, bs, pt_req)
     ws_bytes = pkv.decode_workspace_bytes(B, Hq, Hkv, D, MB, bs, pt_req)
-    ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
     out = torch.empty_like(d["query"])
     launches_per_step = 2 + (1 if plan_np > 1 else 0)
     stream = torch.cuda.current_stream(dev)
+    cascade = args.cascade == "on" or (args.cascade == "auto" and cfg.shared_prefix > 0)
+    if cascade:
+        cas = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in
+               workloads.cascade_inputs(step, cfg.shared_prefix, cfg.samples).items()}
+        ws_bytes = int(pkv.lib().pkv_decode_cascade_workspace_bytes(
+            B, Hq, Hkv, D, cas["prefix_tables"].shape[1], cas["suffix_tables"].shape[1],
+            cas["max_group_size"], bs, pt_req))
+        launches_per_step = 4
+    ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
+
+    def decode_call(query, tables, lens):
+        if cascade:
+            return pkv.paged_attention_decode_cascade(
+                query, d["key_cache"], d["value_cache"], cas["prefix_tables"], cas["prefix_lens"],
+                cas["group_start"], cas["suffix_tables"], cas["suffix_lens"], d["scale"],
+                max_group_size=cas["max_group_size"], partition_tokens=pt_req, out=out,
+                workspace=ws)
+        return pkv.paged_attention_decode(query, d["key_cache"], d["value_cache"], tables, lens,
+                                          d["scale"], partition_tokens=pt_req, out=out,
+                                          workspace=ws)
 
     def one_step():
         pkv.kv_cache_write(d["new_key"], d["new_value"], d["slot_mapping"], d["key_cache"],
                            d["value_cache"])
-        pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
-                                   d["context_lens"], d["scale"], partition_tokens=pt_req,
-                                   out=out, workspace=ws)
+        decode_call(d["query"], d["block_tables"], d["context_lens"])
 
     pkv.device_flags(clear=True)
     for _ in range(args.warmup):
@@ -367,9 +384,7 @@ def run_gpu(args, cfg, world, rank, local):
     torch.cuda.synchronize()
     for i in range(Kd):
         ev[i][0].record(stream)
-        pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"], d["block_tables"],
-                                   d["context_lens"], d["scale"], partition_tokens=pt_req,
-                                   out=out, workspace=ws)
+        decode_call(d["query"], d["block_tables"], d["context_lens"])
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     decode_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)   # decode (+ merge) per call
@@ -390,9 +405,7 @@ def run_gpu(args, cfg, world, rank, local):
                 dev_in[k].copy_(v, non_blocking=True)
             pkv.kv_cache_write(dev_in["new_key"], dev_in["new_value"], dev_in["slot_mapping"],
                                d["key_cache"], d["value_cache"])
-            pkv.paged_attention_decode(dev_in["query"], d["key_cache"], d["value_cache"],
-                                       dev_in["block_tables"], dev_in["context_lens"], d["scale"],
-                                       partition_tokens=pt_req, out=out, workspace=ws)
+            decode_call(dev_in["query"], dev_in["block_tables"], dev_in["context_lens"])
             host_out.copy_(out, non_blocking=True)
             stream.synchronize()                       # the caller reads the result
 
@@ -410,12 +423,13 @@ def run_gpu(args, cfg, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
-        e2e_gbs = sum_over_ranks(nbytes["decode"] + nbytes["write"], world) / (e2e_ms * 1e-3) / 1e9
+        e2e_gbs = sum_over_ranks(nbytes["decode_unique"] + nbytes["write"], world) / (e2e_ms * 1e-3) / 1e9
         e2e = {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": Ke,
                "tokens_per_s": round(sum_over_ranks(B, world) / (e2e_ms * 1e-3), 1)}
 
-    value, ms_step = job_throughput(nbytes["decode"] + nbytes["write"], ms_total / K, world)
+    # unique bytes: a block shared by several sequences' tables counts once
+    value, ms_step = job_throughput(nbytes["decode_unique"] + nbytes["write"], ms_total / K, world)
     # every collective before any rank-0-only code: all ranks take the same steps
     tokens = sum_over_ranks(B, world)
     kv_tokens_all = sum_over_ranks(nbytes["kv_tokens"], world)
@@ -428,7 +442,9 @@ def run_gpu(args, cfg, world, rank, local):
                 "traffic": committed_traffic(cfg.name),
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6650 GB/s",
-                "kernel": "paged_decode_kernel" + (" + lse_merge_kernel" if plan_np > 1 else ""),
+                "kernel": ("prefix_decode_kernel + paged_decode_kernel (suffixes) + "
+                           "lse_merge_cascade_kernel" if cascade else
+                           "paged_decode_kernel" + (" + lse_merge_kernel" if plan_np > 1 else "")),
                 "bytes_per_launch": nbytes["decode_unique"], "launch_ms": round(decode_ms, 5),
                 "frac_of_8000": round(achieved / 8000.0, 4)}
 
@@ -452,6 +468,7 @@ def run_gpu(args, cfg, world, rank, local):
                        "num_blocks": NB, "max_blocks": MB,
                        "context_tokens": nbytes["kv_tokens"],
                        "partition_tokens": plan_pt, "num_partitions": plan_np,
+                       "cascade": cascade,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": (f"inputs larger than L2: {nbytes['kv_unique'] / 1e6:.0f} MB of K/V "
                               f"per step vs 126 MB L2, no flush")
@@ -490,6 +507,8 @@ def main(argv=None):
     ap.add_argument("--roofline-launches", type=int, default=500)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
+    ap.add_argument("--cascade", default="auto", choices=["auto", "on", "off"],
+                    help="shared-prefix decode (auto: for workloads with a shared prefix)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")

@@ -171,6 +171,46 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
                                       pkv_dtype dtype, void *stream);
 
 /*
+ * paged_attention_decode_cascade -- decode for sequences that share a prefix
+ * ([FC] 二.3: parallel samples and beams share the prompt's blocks; [YK] 三
+ * for the block walk).  The result equals pkv_paged_attention_decode over the
+ * concatenated tables, but each shared prefix block is read from HBM once
+ * per group instead of once per sequence.
+ *
+ *   prefix_tables  [num_groups, max_prefix_blocks] int32   device, read
+ *   prefix_lens    [num_groups] int32, multiples of block_size, device, read
+ *   group_start    [num_groups + 1] int32: group g owns sequences
+ *                  group_start[g] .. group_start[g+1]-1 (ascending,
+ *                  at most max_group_size each)          device, read
+ *   suffix_tables  [batch, max_suffix_blocks] int32: each sequence's own
+ *                  blocks, the tokens after its group's prefix    device, read
+ *   suffix_lens    [batch] int32 (0 allowed)              device, read
+ *   workspace      pkv_decode_cascade_workspace_bytes(...) bytes, 256-byte
+ *                  aligned (partial records of prefix and suffix passes)
+ *
+ * Sequence b attends over prefix_tables[g] (prefix_lens[g] tokens) followed by
+ * suffix_tables[b] (suffix_lens[b] tokens); sequences outside every group
+ * attend over their suffix only.  Three kernels: the prefix pass (a producer
+ * warp streams each prefix block into a shared-memory ring, consumer warps
+ * apply all of the group's query rows to it), the regular decode over the
+ * suffixes writing partial records, and a log-sum-exp merge of both.
+ * partition_tokens as for pkv_decode_plan (0: 512-token partitions).  Invalid
+ * group bounds or prefix lengths set PKV_DEVFLAG_CONTEXT_RANGE.
+ */
+size_t pkv_decode_cascade_workspace_bytes(int batch, int num_heads, int num_kv_heads, int head_dim,
+                                          int max_prefix_blocks, int max_suffix_blocks,
+                                          int max_group_size, int block_size,
+                                          int partition_tokens);
+pkv_status pkv_paged_attention_decode_cascade(
+    const void *query, const void *key_cache, const void *value_cache,
+    const int32_t *prefix_tables, int max_prefix_blocks, const int32_t *prefix_lens,
+    const int32_t *group_start, int num_groups, int max_group_size,
+    const int32_t *suffix_tables, int max_suffix_blocks, const int32_t *suffix_lens, int batch,
+    int num_heads, int num_kv_heads, int head_dim, int block_size, int64_t num_blocks,
+    float scale, int partition_tokens, void *workspace, size_t workspace_bytes, void *out,
+    pkv_dtype dtype, void *stream);
+
+/*
  * paged_attention_decode_static_workspace -- the same decode as
  * pkv_paged_attention_decode, for callers that cannot allocate device memory
  * at call time (an allocator that owns the whole pool, a serving runtime that

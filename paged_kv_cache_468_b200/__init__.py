@@ -17,6 +17,7 @@ from .pagedkv import (  # noqa: F401
     kv_cache_write,
     lib,
     paged_attention_decode,
+    paged_attention_decode_cascade,
     selftest_bounded_wait,
     version,
 )

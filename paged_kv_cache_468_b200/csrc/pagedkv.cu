@@ -40,6 +40,8 @@ pkv_status cuda_fail(cudaError_t e, const char *what)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
 constexpr int kPlanSmCount = 148;        // B200 SM count used by the automatic plan
 constexpr int kAutoPartitionTokens = 512;
 
@@ -429,6 +431,7 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
     a.num_blocks = (int)num_blocks;
     a.part_tokens = pt;
     a.num_parts = np;
+    a.records_only = 0;
     a.scale_log2 = (float)((double)scale * 1.4426950408889634);
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -451,6 +454,216 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Cascade decode (shared prefixes)
+// ---------------------------------------------------------------------------
+namespace {
+
+struct CascadePlan {
+    int pt;        // partition length in tokens (prefix and suffix)
+    int pp;        // prefix partitions
+    int ps;        // suffix partitions
+    int nwq;       // consumer warps per prefix CTA
+    int chunks;    // member chunks per group
+    size_t m_p, l_p, o_p, m_s, l_s, o_s, total;   // workspace offsets
+};
+
+pkv_status cascade_plan(int batch, int Hq, int Hkv, int D, int max_prefix_blocks,
+                        int max_suffix_blocks, int max_group_size, int bs, int partition_tokens,
+                        CascadePlan *c)
+{
+    pkv_status s = check_shapes(batch, Hq, Hkv, D, std::max(1, max_suffix_blocks), bs);
+    if (s != PKV_OK)
+        return s;
+    if (max_prefix_blocks <= 0 || max_suffix_blocks <= 0 || max_group_size <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "max_prefix_blocks, max_suffix_blocks and max_group_size "
+                    "must be positive");
+    if ((int64_t)max_prefix_blocks * bs >= ((int64_t)1 << 30))
+        return fail(PKV_ERR_INVALID_ARG, "max_prefix_blocks * block_size too large");
+    c->pt = partition_tokens > 0 ? (partition_tokens + bs - 1) / bs * bs : kAutoPartitionTokens;
+    c->pp = (max_prefix_blocks * bs + c->pt - 1) / c->pt;
+    c->ps = (max_suffix_blocks * bs + c->pt - 1) / c->pt;
+    const int rows = max_group_size * (Hq / Hkv);
+    c->nwq = rows <= 8 ? 1 : (rows <= 16 ? 2 : (rows <= 32 ? 4 : 8));
+    c->chunks = (rows + c->nwq * 8 - 1) / (c->nwq * 8);
+    const size_t rp = (size_t)batch * Hq * c->pp, rs = (size_t)batch * Hq * c->ps;
+    c->m_p = 0;
+    c->l_p = align256(c->m_p + rp * 4);
+    c->o_p = align256(c->l_p + rp * 4);
+    c->m_s = align256(c->o_p + rp * (size_t)D * 4);
+    c->l_s = align256(c->m_s + rs * 4);
+    c->o_s = align256(c->l_s + rs * 4);
+    c->total = align256(c->o_s + rs * (size_t)D * 4);
+    return PKV_OK;
+}
+
+template <int D, int BS, bool BF16, int NWQ>
+cudaError_t launch_prefix(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::CascadeArgs &c,
+                          cudaStream_t st)
+{
+    constexpr int S = BS == 16 ? 4 : 3;
+    using Shape = pkv::DecodeShape<D, BS, 1, S>;
+    constexpr int smem = S * Shape::kStageBytes + 1024;
+    auto kern = pkv::prefix_decode_kernel<D, BS, BF16, NWQ, S>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    const dim3 grid((unsigned)c.num_parts, (unsigned)c.num_kv_heads,
+                    (unsigned)((size_t)c.num_groups * c.chunks));
+    return launch_pdl(kern, grid, dim3((NWQ + 1) * 32), smem, st, mk, mv, c);
+}
+
+template <int D, int BS, bool BF16>
+cudaError_t dispatch_prefix_nwq(int nwq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                const pkv::CascadeArgs &c, cudaStream_t st)
+{
+    switch (nwq) {
+    case 1: return launch_prefix<D, BS, BF16, 1>(mk, mv, c, st);
+    case 2: return launch_prefix<D, BS, BF16, 2>(mk, mv, c, st);
+    case 4: return launch_prefix<D, BS, BF16, 4>(mk, mv, c, st);
+    default: return launch_prefix<D, BS, BF16, 8>(mk, mv, c, st);
+    }
+}
+
+template <bool BF16>
+cudaError_t dispatch_prefix(int D, int bs, int nwq, const CUtensorMap &mk, const CUtensorMap &mv,
+                            const pkv::CascadeArgs &c, cudaStream_t st)
+{
+    if (D == 64 && bs == 16) return dispatch_prefix_nwq<64, 16, BF16>(nwq, mk, mv, c, st);
+    if (D == 64 && bs == 32) return dispatch_prefix_nwq<64, 32, BF16>(nwq, mk, mv, c, st);
+    if (D == 128 && bs == 16) return dispatch_prefix_nwq<128, 16, BF16>(nwq, mk, mv, c, st);
+    return dispatch_prefix_nwq<128, 32, BF16>(nwq, mk, mv, c, st);
+}
+
+}  // namespace
+
+extern "C" size_t pkv_decode_cascade_workspace_bytes(int batch, int num_heads, int num_kv_heads,
+                                                     int head_dim, int max_prefix_blocks,
+                                                     int max_suffix_blocks, int max_group_size,
+                                                     int block_size, int partition_tokens)
+{
+    CascadePlan c;
+    if (cascade_plan(batch, num_heads, num_kv_heads, head_dim, max_prefix_blocks, max_suffix_blocks,
+                     max_group_size, block_size, partition_tokens, &c) != PKV_OK)
+        return 0;
+    return c.total;
+}
+
+extern "C" pkv_status pkv_paged_attention_decode_cascade(
+    const void *query, const void *key_cache, const void *value_cache, const int32_t *prefix_tables,
+    int max_prefix_blocks, const int32_t *prefix_lens, const int32_t *group_start, int num_groups,
+    int max_group_size, const int32_t *suffix_tables, int max_suffix_blocks,
+    const int32_t *suffix_lens, int batch, int num_heads, int num_kv_heads, int head_dim,
+    int block_size, int64_t num_blocks, float scale, int partition_tokens, void *workspace,
+    size_t workspace_bytes, void *out, pkv_dtype dtype, void *stream)
+{
+    CascadePlan plan;
+    pkv_status s = cascade_plan(batch, num_heads, num_kv_heads, head_dim, max_prefix_blocks,
+                                max_suffix_blocks, max_group_size, block_size, partition_tokens, &plan);
+    if (s != PKV_OK)
+        return s;
+    if (dtype != PKV_F16 && dtype != PKV_BF16)
+        return fail(PKV_ERR_INVALID_ARG, "dtype %d", (int)dtype);
+    if (num_groups < 0 || num_groups > batch)
+        return fail(PKV_ERR_INVALID_ARG, "num_groups %d (0 .. batch)", num_groups);
+    if (num_blocks <= 0 || num_blocks * block_size >= ((int64_t)1 << 31))
+        return fail(PKV_ERR_INVALID_ARG, "num_blocks %lld: need 0 < num_blocks*block_size < 2^31",
+                    (long long)num_blocks);
+    if (!std::isfinite(scale))
+        return fail(PKV_ERR_INVALID_ARG, "scale is not finite");
+    if (batch == 0)
+        return PKV_OK;
+    if (!query || !key_cache || !value_cache || !suffix_tables || !suffix_lens || !out ||
+        (num_groups > 0 && (!prefix_tables || !prefix_lens || !group_start)))
+        return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
+        return fail(PKV_ERR_MISALIGNED, "query/cache/out pointers must be 16-byte aligned");
+    if (!workspace || workspace_bytes < plan.total)
+        return fail(PKV_ERR_WORKSPACE, "workspace of %zu bytes needed, %zu given", plan.total,
+                    workspace ? workspace_bytes : (size_t)0);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(PKV_ERR_MISALIGNED, "workspace must be 256-byte aligned");
+
+    CUtensorMap mk, mv;
+    if ((s = make_cache_map(&mk, key_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
+        return s;
+    if ((s = make_cache_map(&mv, value_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
+        return s;
+    unsigned char *ws = static_cast<unsigned char *>(workspace);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float scale_log2 = (float)((double)scale * 1.4426950408889634);
+
+    // level 1: shared prefixes, one pass per group
+    pkv::CascadeArgs c;
+    c.query = static_cast<const uint16_t *>(query);
+    c.prefix_tables = prefix_tables;
+    c.prefix_lens = prefix_lens;
+    c.group_start = group_start;
+    c.rec_m = reinterpret_cast<float *>(ws + plan.m_p);
+    c.rec_l = reinterpret_cast<float *>(ws + plan.l_p);
+    c.rec_o = reinterpret_cast<float *>(ws + plan.o_p);
+    c.batch = batch;
+    c.max_prefix_blocks = max_prefix_blocks;
+    c.num_groups = num_groups;
+    c.max_group_size = max_group_size;
+    c.num_heads = num_heads;
+    c.num_kv_heads = num_kv_heads;
+    c.group = num_heads / num_kv_heads;
+    c.num_blocks = (int)num_blocks;
+    c.part_tokens = plan.pt;
+    c.num_parts = plan.pp;
+    c.chunks = plan.chunks;
+    c.scale_log2 = scale_log2;
+    cudaError_t e = cudaSuccess;
+    if (num_groups > 0) {
+        e = dtype == PKV_BF16 ? dispatch_prefix<true>(head_dim, block_size, plan.nwq, mk, mv, c, st)
+                              : dispatch_prefix<false>(head_dim, block_size, plan.nwq, mk, mv, c, st);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "prefix_decode_kernel launch");
+    }
+
+    // level 2: each sequence's own blocks, as partition records
+    pkv::DecodeArgs a;
+    a.query = c.query;
+    a.block_tables = suffix_tables;
+    a.context_lens = suffix_lens;
+    a.out = static_cast<uint16_t *>(out);
+    a.ws_m = reinterpret_cast<float *>(ws + plan.m_s);
+    a.ws_l = reinterpret_cast<float *>(ws + plan.l_s);
+    a.ws_o = reinterpret_cast<float *>(ws + plan.o_s);
+    a.max_blocks = max_suffix_blocks;
+    a.num_heads = num_heads;
+    a.group = num_heads / num_kv_heads;
+    a.num_blocks = (int)num_blocks;
+    a.part_tokens = plan.ps > 1 ? plan.pt : max_suffix_blocks * block_size;
+    a.num_parts = plan.ps;
+    a.records_only = 1;
+    a.scale_log2 = scale_log2;
+    s = dtype == PKV_BF16 ? dispatch_decode<true>(head_dim, block_size, mk, mv, a, batch, num_kv_heads, st)
+                          : dispatch_decode<false>(head_dim, block_size, mk, mv, a, batch, num_kv_heads, st);
+    if (s != PKV_OK)
+        return s;
+
+    // merge prefix and suffix records of every (sequence, query head) row
+    constexpr int NT = 512;
+    const int rows = batch * num_heads;
+    const int suffix_span = max_suffix_blocks * block_size;
+    auto go = [&](auto kern, int D) {
+        const int ng = NT / D;
+        return launch_pdl(kern, dim3((unsigned)((rows + ng - 1) / ng)), dim3(NT), 0, st, c, a.ws_m,
+                          a.ws_l, a.ws_o, suffix_lens, plan.ps, a.part_tokens, suffix_span, a.out);
+    };
+    if (dtype == PKV_BF16)
+        e = head_dim == 64 ? go(pkv::lse_merge_cascade_kernel<true, 64, NT>, 64)
+                           : go(pkv::lse_merge_cascade_kernel<true, 128, NT>, 128);
+    else
+        e = head_dim == 64 ? go(pkv::lse_merge_cascade_kernel<false, 64, NT>, 64)
+                           : go(pkv::lse_merge_cascade_kernel<false, 128, NT>, 128);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "lse_merge_cascade_kernel launch");
+    return PKV_OK;
+}
 
 // ---------------------------------------------------------------------------
 // Decode with a library-owned workspace (no allocation by anyone at call time)

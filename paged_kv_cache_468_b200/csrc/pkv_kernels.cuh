@@ -122,6 +122,130 @@ __global__ void kv_write_kernel(const uint4 *__restrict__ key, const uint4 *__re
 }
 
 // ---------------------------------------------------------------------------
+// One K/V block of the group tile, for one warp
+// ---------------------------------------------------------------------------
+// sk / sv: shared addresses of the swizzled K and V tiles of one block (BS
+// token rows of D columns, 64-column halves of BS*128 bytes, 128-byte
+// swizzle); valid: rows holding tokens (later rows are masked; their V rows
+// must be zero).  qf: Q^T fragments of this warp's 8 query columns.  Updates
+// the running max m_run / lane-partial normaliser l_run of the lane's columns
+// 2c, 2c+1 (base-2 units) and the O^T accumulators (high part and remainder of
+// P, each times V):
+//   S^T[t, n] = sum_d K[t, d] Q[n, d]            (mma.sync m16n8k16, fp32)
+//   online softmax per column n
+//   O^T[d, n] += sum_t V[t, d] P[t, n]
+template <int D, int BS, bool BF16>
+__device__ __forceinline__ void attend_block(uint32_t sk, uint32_t sv, int valid,
+                                             const uint32_t (&qf)[D / 16][2], float scale_log2,
+                                             float (&m_run)[2], float (&l_run)[2],
+                                             float (&acc_hi)[D / 16][4], float (&acc_lo)[D / 16][4],
+                                             int lane)
+{
+    constexpr int MT = BS / 16;
+    constexpr int KS = D / 16;
+    constexpr int kHalfBytes = BS * 128;
+    // ---- scores: S^T[t, n] = sum_d K[t, d] Q[n, d] ----
+    float sc[MT][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        float s0[4] = {0.f, 0.f, 0.f, 0.f};   // two accumulation chains (even / odd k)
+        float s1[4] = {0.f, 0.f, 0.f, 0.f};
+        const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            const int chunk = (ks & 3) * 2 + (lane >> 4);
+            const uint32_t addr = sk + (uint32_t)((ks >> 2) * kHalfBytes + row * 128 +
+                                                  ((chunk ^ (row & 7)) << 4));
+            uint32_t af[4];
+            ldsm_x4(addr, af);
+            if (ks & 1)
+                mma_16816<BF16>(s1, af, qf[ks][0], qf[ks][1]);
+            else
+                mma_16816<BF16>(s0, af, qf[ks][0], qf[ks][1]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            sc[mt][i] = s0[i] + s1[i];
+    }
+
+    // ---- online softmax (base 2), per column n = 2c + j ----
+    float mx[2] = {kNegInf, kNegInf};
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int t = mt * 16 + (lane >> 2) + (i >= 2 ? 8 : 0);
+            const float v = t < valid ? sc[mt][i] * scale_log2 : kNegInf;
+            sc[mt][i] = v;
+            mx[i & 1] = fmaxf(mx[i & 1], v);
+        }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 4));
+        mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
+        mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
+    }
+    float alpha[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float mnew = fmaxf(m_run[j], mx[j]);
+        alpha[j] = ex2(m_run[j] - mnew);   // 0 on the first block (m_run = -inf)
+        m_run[j] = mnew;
+    }
+    float ls[2] = {0.f, 0.f};
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float p = ex2(sc[mt][i] - m_run[i & 1]);
+            sc[mt][i] = p;
+            ls[i & 1] += p;
+        }
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+        l_run[j] = l_run[j] * alpha[j] + ls[j];
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt) {
+        acc_hi[dt][0] *= alpha[0];
+        acc_hi[dt][1] *= alpha[1];
+        acc_hi[dt][2] *= alpha[0];
+        acc_hi[dt][3] *= alpha[1];
+        acc_lo[dt][0] *= alpha[0];
+        acc_lo[dt][1] *= alpha[1];
+        acc_lo[dt][2] *= alpha[0];
+        acc_lo[dt][3] *= alpha[1];
+    }
+
+    // ---- O^T[d, n] += sum_t V[t, d] P[t, n] ----
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const uint32_t h01 = pack2<BF16>(sc[mt][0], sc[mt][1]);
+        const uint32_t h23 = pack2<BF16>(sc[mt][2], sc[mt][3]);
+        const float2 f01 = unpack2<BF16>(h01);
+        const float2 f23 = unpack2<BF16>(h23);
+        const uint32_t l01 = pack2<BF16>(sc[mt][0] - f01.x, sc[mt][1] - f01.y);
+        const uint32_t l23 = pack2<BF16>(sc[mt][2] - f23.x, sc[mt][3] - f23.y);
+        const uint32_t bh0 = movmatrix_trans(h01);
+        const uint32_t bh1 = movmatrix_trans(h23);
+        const uint32_t bl0 = movmatrix_trans(l01);
+        const uint32_t bl1 = movmatrix_trans(l23);
+        const int t = mt * 16 + (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt) {
+            const int d = dt * 16 + ((lane >> 3) & 1) * 8;
+            const int chunk = (d & 63) >> 3;
+            const uint32_t addr = sv + (uint32_t)((d >> 6) * kHalfBytes + t * 128 +
+                                                  ((chunk ^ (t & 7)) << 4));
+            uint32_t af[4];
+            ldsm_x4_trans(addr, af);
+            mma_16816<BF16>(acc_hi[dt], af, bh0, bh1);
+            mma_16816<BF16>(acc_lo[dt], af, bl0, bl1);
+        }
+    }
+
+}
+
+// ---------------------------------------------------------------------------
 // Decode
 // ---------------------------------------------------------------------------
 struct DecodeArgs {
@@ -138,6 +262,7 @@ struct DecodeArgs {
     int num_blocks;
     int part_tokens;              // tokens per partition (multiple of block size)
     int num_parts;                // partitions per sequence (1 = single pass)
+    int records_only;             // 1: write partition records even for one partition
     float scale_log2;             // scale * log2(e)
 };
 
@@ -178,7 +303,7 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int lane = threadIdx.x & 31;
     const int Hq = a.num_heads;
     const int G = a.group;
-    const bool split = a.num_parts > 1;
+    const bool split = a.num_parts > 1 || a.records_only;
 
     // Set-up that touches no global memory, then wait for the previous kernel
     // on the stream (programmatic dependent launch lets this CTA start while
@@ -327,104 +452,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             __syncwarp();
         }
 
-        // ---- scores: S^T[t, n] = sum_d K[t, d] Q[n, d] ----
-        float sc[MT][4];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            float s0[4] = {0.f, 0.f, 0.f, 0.f};   // two accumulation chains (even / odd k)
-            float s1[4] = {0.f, 0.f, 0.f, 0.f};
-            const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-                const int chunk = (ks & 3) * 2 + (lane >> 4);
-                const uint32_t addr = sk + (uint32_t)((ks >> 2) * kHalfBytes + row * 128 +
-                                                      ((chunk ^ (row & 7)) << 4));
-                uint32_t af[4];
-                ldsm_x4(addr, af);
-                if (ks & 1)
-                    mma_16816<BF16>(s1, af, qf[ks][0], qf[ks][1]);
-                else
-                    mma_16816<BF16>(s0, af, qf[ks][0], qf[ks][1]);
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                sc[mt][i] = s0[i] + s1[i];
-        }
-
-        // ---- online softmax (base 2), per column n = 2c + j ----
-        float mx[2] = {kNegInf, kNegInf};
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int t = mt * 16 + (lane >> 2) + (i >= 2 ? 8 : 0);
-                const float v = t < valid ? sc[mt][i] * a.scale_log2 : kNegInf;
-                sc[mt][i] = v;
-                mx[i & 1] = fmaxf(mx[i & 1], v);
-            }
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 4));
-            mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
-            mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
-        }
-        float alpha[2];
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const float mnew = fmaxf(m_run[j], mx[j]);
-            alpha[j] = ex2(m_run[j] - mnew);   // 0 on the first block (m_run = -inf)
-            m_run[j] = mnew;
-        }
-        float ls[2] = {0.f, 0.f};
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const float p = ex2(sc[mt][i] - m_run[i & 1]);
-                sc[mt][i] = p;
-                ls[i & 1] += p;
-            }
-#pragma unroll
-        for (int j = 0; j < 2; ++j)
-            l_run[j] = l_run[j] * alpha[j] + ls[j];
-#pragma unroll
-        for (int dt = 0; dt < KS; ++dt) {
-            acc_hi[dt][0] *= alpha[0];
-            acc_hi[dt][1] *= alpha[1];
-            acc_hi[dt][2] *= alpha[0];
-            acc_hi[dt][3] *= alpha[1];
-            acc_lo[dt][0] *= alpha[0];
-            acc_lo[dt][1] *= alpha[1];
-            acc_lo[dt][2] *= alpha[0];
-            acc_lo[dt][3] *= alpha[1];
-        }
-
-        // ---- O^T[d, n] += sum_t V[t, d] P[t, n] ----
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const uint32_t h01 = pack2<BF16>(sc[mt][0], sc[mt][1]);
-            const uint32_t h23 = pack2<BF16>(sc[mt][2], sc[mt][3]);
-            const float2 f01 = unpack2<BF16>(h01);
-            const float2 f23 = unpack2<BF16>(h23);
-            const uint32_t l01 = pack2<BF16>(sc[mt][0] - f01.x, sc[mt][1] - f01.y);
-            const uint32_t l23 = pack2<BF16>(sc[mt][2] - f23.x, sc[mt][3] - f23.y);
-            const uint32_t bh0 = movmatrix_trans(h01);
-            const uint32_t bh1 = movmatrix_trans(h23);
-            const uint32_t bl0 = movmatrix_trans(l01);
-            const uint32_t bl1 = movmatrix_trans(l23);
-            const int t = mt * 16 + (lane & 7) + (lane >> 4) * 8;
-#pragma unroll
-            for (int dt = 0; dt < KS; ++dt) {
-                const int d = dt * 16 + ((lane >> 3) & 1) * 8;
-                const int chunk = (d & 63) >> 3;
-                const uint32_t addr = sv + (uint32_t)((d >> 6) * kHalfBytes + t * 128 +
-                                                      ((chunk ^ (t & 7)) << 4));
-                uint32_t af[4];
-                ldsm_x4_trans(addr, af);
-                mma_16816<BF16>(acc_hi[dt], af, bh0, bh1);
-                mma_16816<BF16>(acc_lo[dt], af, bl0, bl1);
-            }
-        }
+        attend_block<D, BS, BF16>(sk, sv, valid, qf, a.scale_log2, m_run, l_run, acc_hi, acc_lo,
+                                  lane);
 
         __syncwarp();
         if (k + S < nk) {
@@ -497,6 +526,291 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             }
         }
     }
+}
+
+// ---------------------------------------------------------------------------
+// Cascade decode, level 1: a shared prefix read once for a whole group
+// ---------------------------------------------------------------------------
+// Parallel samples of one prompt share the prompt's blocks ("23.1 vLLM：高吞吐
+// 推理框架原理与部署", section 二.3).  Sequences group_start[g] ..
+// group_start[g+1]-1 share the prefix_lens[g] tokens (a multiple of the block
+// size) listed in prefix_tables[g].  One CTA per (prefix partition, kv head,
+// group member chunk): a producer warp streams the partition's K/V blocks
+// through a CTA-wide ring of S stages (TMA, full/empty mbarriers), and each
+// of NWQ consumer warps applies 8 of the group's query rows (member, head of
+// the GQA group) to every tile, so each prefix block is read from HBM once per
+// group instead of once per sequence.  Each consumer writes, per query row,
+// the partition's record (max, normaliser, normalised row); level 2 (the
+// decode kernel over each sequence's own suffix, records only) and the
+// cascade merge complete the result, which equals the decode over the
+// concatenated table.
+struct CascadeArgs {
+    const uint16_t *query;           // [B, Hq, D]
+    const int32_t *prefix_tables;    // [num_groups, max_prefix_blocks]
+    const int32_t *prefix_lens;      // [num_groups]
+    const int32_t *group_start;      // [num_groups + 1]
+    float *rec_m;                    // prefix records [B*Hq, num_parts]
+    float *rec_l;
+    float *rec_o;                    // [B*Hq, num_parts, D]
+    int batch;
+    int max_prefix_blocks;
+    int num_groups;
+    int max_group_size;
+    int num_heads;
+    int num_kv_heads;
+    int group;                       // Hq / Hkv
+    int num_blocks;
+    int part_tokens;                 // prefix partition length (multiple of BS)
+    int num_parts;                   // prefix partitions
+    int chunks;                      // member chunks per group
+    float scale_log2;
+};
+
+template <int D, int BS, bool BF16, int NWQ, int S>
+__global__ void __launch_bounds__((NWQ + 1) * 32, 1)
+prefix_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                     const CascadeArgs a)
+{
+    using Shape = DecodeShape<D, BS, 1, S>;
+    constexpr int kHalfBytes = Shape::kHalfBytes;
+    constexpr int kTileBytes = Shape::kTileBytes;
+    constexpr int kStageBytes = Shape::kStageBytes;
+    constexpr int KS = D / 16;
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ __align__(8) uint64_t full[S];
+    __shared__ __align__(8) uint64_t empty[S];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const uint32_t ring_s = smem_addr(smem);
+
+    const int pp = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int g = blockIdx.z / a.chunks;
+    const int mc = blockIdx.z - g * a.chunks;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = a.group;
+
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_addr(&full[s]), 1);
+            mbar_init(smem_addr(&empty[s]), NWQ);
+        }
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    fence_mbar_init();
+    __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    int first = __ldg(a.group_start + g);
+    int count = __ldg(a.group_start + g + 1) - first;
+    if (first < 0 || count < 0 || first + count > a.batch || count > a.max_group_size) {
+        if (threadIdx.x == 0 && pp == 0 && kvh == 0 && mc == 0)
+            raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+        first = first < 0 ? 0 : (first > a.batch ? a.batch : first);
+        count = count < 0 ? 0 : count;
+        count = min(count, min(a.max_group_size, a.batch - first));
+    }
+    const int row0 = mc * NWQ * 8;                  // first query row of this chunk
+    const int nrows = min(NWQ * 8, count * G - row0);
+    int Lp = __ldg(a.prefix_lens + g);
+    const int span = a.max_prefix_blocks * BS;
+    if (Lp < 0 || Lp > span || Lp % BS != 0) {
+        if (threadIdx.x == 0 && pp == 0 && kvh == 0 && mc == 0)
+            raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+        Lp = Lp < 0 ? 0 : (Lp > span ? span : Lp - Lp % BS);
+    }
+    const int tok0 = pp * a.part_tokens;
+    const int tok1 = min(Lp, tok0 + a.part_tokens);
+    if (nrows <= 0 || tok1 <= tok0)
+        return;                                     // nothing here (the merge skips it)
+    const int nblk = (tok1 - tok0) / BS;
+    const int blk0 = tok0 / BS;
+
+    if (warp == NWQ) {
+        // ---- producer: one block per stage, S ahead of the consumers ----
+        const int32_t *trow = a.prefix_tables + (size_t)g * a.max_prefix_blocks + blk0;
+        const uint64_t policy = policy_evict_first();
+        int ids = 0;
+        for (int k = 0; k < nblk; ++k) {
+            const int s = k % S;
+            if (k >= S) {
+                const bool ok = mbar_wait_bounded(smem_addr(&empty[s]), (uint32_t)(((k / S) - 1) & 1),
+                                                  kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    if (lane == 0)
+                        raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+                    break;
+                }
+            }
+            if ((k & 31) == 0)
+                ids = k + lane < nblk ? __ldg(trow + k + lane) : 0;
+            int blk = __shfl_sync(0xffffffffu, ids, k & 31);
+            if ((unsigned)blk >= (unsigned)a.num_blocks) {
+                if (lane == 0)
+                    raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
+                blk = 0;
+            }
+            if (lane == 0) {
+                const uint32_t bar = smem_addr(&full[s]);
+                const uint32_t dk = ring_s + (uint32_t)(s * kStageBytes);
+                mbar_arrive_expect_tx(bar, kStageBytes);
+#pragma unroll
+                for (int h = 0; h < Shape::kHalves; ++h) {
+                    tma_load_3d(dk + h * kHalfBytes, &tm_k, bar, h * 64, kvh, blk * BS, policy);
+                    tma_load_3d(dk + kTileBytes + h * kHalfBytes, &tm_v, bar, h * 64, kvh, blk * BS,
+                                policy);
+                }
+            }
+        }
+        return;
+    }
+
+    // ---- consumers: warp w owns query rows row0 + 8w + n, n = 0..7 ----
+    uint32_t qf[KS][2];
+    const int n_own = lane >> 2;
+    const int r_own = row0 + warp * 8 + n_own;       // query row of column n_own
+    const bool col_ok = r_own < row0 + nrows;
+    {
+        const int member = r_own / G;
+        const int gq = r_own - member * G;
+        const int c = lane & 3;
+        const uint32_t *q32 = reinterpret_cast<const uint32_t *>(
+            a.query + ((size_t)(first + (col_ok ? member : 0)) * a.num_heads + (size_t)kvh * G +
+                       (col_ok ? gq : 0)) * D);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+            qf[ks][0] = col_ok ? __ldg(q32 + ks * 8 + c) : 0u;
+            qf[ks][1] = col_ok ? __ldg(q32 + ks * 8 + 4 + c) : 0u;
+        }
+    }
+    float m_run[2] = {kNegInf, kNegInf};
+    float l_run[2] = {0.f, 0.f};
+    float acc_hi[KS][4], acc_lo[KS][4];
+#pragma unroll
+    for (int dt = 0; dt < KS; ++dt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            acc_hi[dt][i] = 0.f;
+            acc_lo[dt][i] = 0.f;
+        }
+    int consumed = 0;
+    for (int k = 0; k < nblk; ++k) {
+        const int s = k % S;
+        const bool got = mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((k / S) & 1), kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+            if (lane == 0)
+                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+            break;
+        }
+        consumed = k + 1;
+        const uint32_t sk = ring_s + (uint32_t)(s * kStageBytes);
+        attend_block<D, BS, BF16>(sk, sk + kTileBytes, BS, qf, a.scale_log2, m_run, l_run, acc_hi,
+                                  acc_lo, lane);
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(smem_addr(&empty[s]));      // this warp is done with the stage
+    }
+    // stages the producer filled but this warp did not consume (a wait gave up)
+    for (int k = consumed; k < nblk && k < consumed + S; ++k)
+        mbar_wait_bounded(smem_addr(&full[k % S]), (uint32_t)((k / S) & 1), kWaitLimitNs / 8);
+
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 4);
+        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 8);
+        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 16);
+    }
+    // records of the lane's columns 2c, 2c+1
+    const int c = lane & 3;
+    const int r = lane >> 2;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int n = 2 * c + j;
+        const int row_local = row0 + warp * 8 + n;
+        if (row_local >= row0 + nrows)
+            continue;
+        const int member = row_local / G;
+        const int gq = row_local - member * G;
+        const size_t row = (size_t)(first + member) * a.num_heads + (size_t)kvh * G + gq;
+        const size_t rec = row * a.num_parts + pp;
+        const float inv = l_run[j] > 0.f ? 1.f / l_run[j] : 0.f;
+#pragma unroll
+        for (int dt = 0; dt < KS; ++dt) {
+            a.rec_o[rec * D + dt * 16 + r] = (acc_hi[dt][j] + acc_lo[dt][j]) * inv;
+            a.rec_o[rec * D + dt * 16 + r + 8] = (acc_hi[dt][2 + j] + acc_lo[dt][2 + j]) * inv;
+        }
+        if (r == 0) {
+            a.rec_m[rec] = m_run[j];
+            a.rec_l[rec] = l_run[j];
+        }
+    }
+}
+
+// Cascade merge: row (b, h) = its group's prefix records (partitions of the
+// prefix) and its own suffix records (partitions of the suffix), folded by
+// log-sum-exp.  NT threads = NG groups of D, one row per group.
+template <bool BF16, int D, int NT>
+__global__ void __launch_bounds__(NT)
+lse_merge_cascade_kernel(const CascadeArgs c, const float *__restrict__ sm, const float *__restrict__ sl,
+                         const float *__restrict__ so, const int32_t *__restrict__ suffix_lens,
+                         int suffix_parts, int suffix_part_tokens, int suffix_span,
+                         uint16_t *__restrict__ out)
+{
+    constexpr int NG = NT / D;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int d = threadIdx.x % D;
+    const size_t row = (size_t)blockIdx.x * NG + threadIdx.x / D;
+    if (row >= (size_t)c.batch * c.num_heads)
+        return;
+    const int b = (int)(row / c.num_heads);
+    // group of sequence b: the last g with group_start[g] <= b
+    int lo = 0, hi = c.num_groups - 1, g = -1;
+    while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(c.group_start + mid) <= b) {
+            g = mid;
+            lo = mid + 1;
+        } else {
+            hi = mid - 1;
+        }
+    }
+    int np_p = 0;
+    if (g >= 0 && b < __ldg(c.group_start + g + 1)) {
+        int Lp = __ldg(c.prefix_lens + g);
+        Lp = Lp < 0 ? 0 : Lp;
+        np_p = min(c.num_parts, (Lp + c.part_tokens - 1) / c.part_tokens);
+    }
+    int Ls = __ldg(suffix_lens + b);
+    Ls = Ls < 0 ? 0 : (Ls > suffix_span ? suffix_span : Ls);
+    const int np_s = (Ls + suffix_part_tokens - 1) / suffix_part_tokens;
+    float M = kNegInf, den = 0.f, num = 0.f;
+    auto fold = [&](float mp, float lp, float op) {
+        if (!(lp > 0.f))
+            return;
+        if (mp > M) {
+            const float sc = ex2(M - mp);
+            den *= sc;
+            num *= sc;
+            M = mp;
+        }
+        const float w = ex2(mp - M) * lp;
+        den += w;
+        num += w * op;
+    };
+    for (int p = 0; p < np_p; ++p) {
+        const size_t rec = row * c.num_parts + p;
+        fold(__ldg(c.rec_m + rec), __ldg(c.rec_l + rec), __ldg(c.rec_o + rec * D + d));
+    }
+    for (int p = 0; p < np_s; ++p) {
+        const size_t rec = row * suffix_parts + p;
+        fold(__ldg(sm + rec), __ldg(sl + rec), __ldg(so + rec * D + d));
+    }
+    out[row * D + d] = to_storage<BF16>(den > 0.f ? num / den : 0.f);
 }
 
 // ---------------------------------------------------------------------------

@@ -67,6 +67,12 @@ def lib() -> ctypes.CDLL:
         L.pkv_paged_attention_decode.restype = i32
         L.pkv_paged_attention_decode.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                                  f32, i32, P, sz, P, i32, P]
+        L.pkv_decode_cascade_workspace_bytes.restype = sz
+        L.pkv_decode_cascade_workspace_bytes.argtypes = [i32] * 9
+        L.pkv_paged_attention_decode_cascade.restype = i32
+        L.pkv_paged_attention_decode_cascade.argtypes = [
+            P, P, P, P, i32, P, P, i32, i32, P, i32, P, i32, i32, i32, i32, i32, i64, f32, i32, P,
+            sz, P, i32, P]
         L.pkv_alloc_create.restype = P
         L.pkv_alloc_create.argtypes = [i64, i32, u64]
         L.pkv_alloc_destroy.restype = None
@@ -219,6 +225,49 @@ def paged_attention_decode(query: torch.Tensor, key_cache: torch.Tensor, value_c
         bs, NB, float(scale), int(partition_tokens), ws_ptr, ws_bytes, _dev(out, "out"), dt,
         _stream_handle(stream, query.device))
     _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+def paged_attention_decode_cascade(query: torch.Tensor, key_cache: torch.Tensor,
+                                   value_cache: torch.Tensor, prefix_tables: torch.Tensor,
+                                   prefix_lens: torch.Tensor, group_start: torch.Tensor,
+                                   suffix_tables: torch.Tensor, suffix_lens: torch.Tensor,
+                                   scale: float, max_group_size: int, partition_tokens: int = 0,
+                                   out: Optional[torch.Tensor] = None,
+                                   workspace: Optional[torch.Tensor] = None,
+                                   stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Decode with shared prefixes read once per group (see include/pagedkv.h).
+    prefix_tables int32 [G, MPB], prefix_lens int32 [G], group_start int32 [G+1],
+    suffix_tables int32 [B, MSB], suffix_lens int32 [B] -> out [B, Hq, D]."""
+    B, Hq, D = query.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    for name, t, nd in (("prefix_tables", prefix_tables, 2), ("prefix_lens", prefix_lens, 1),
+                        ("group_start", group_start, 1), ("suffix_tables", suffix_tables, 2),
+                        ("suffix_lens", suffix_lens, 1)):
+        if t.dtype != torch.int32 or t.dim() != nd:
+            raise ValueError(f"{name} must be int32 with {nd} dims")
+    G = prefix_tables.shape[0]
+    if prefix_lens.shape != (G,) or group_start.shape != (G + 1,):
+        raise ValueError("prefix_lens must be [num_groups], group_start [num_groups + 1]")
+    if suffix_tables.shape[0] != B or suffix_lens.shape != (B,):
+        raise ValueError("suffix_tables must be [batch, max_suffix_blocks], suffix_lens [batch]")
+    dt = _dtype_code(query)
+    if out is None:
+        out = torch.empty_like(query)
+    MPB, MSB = prefix_tables.shape[1], suffix_tables.shape[1]
+    need = int(lib().pkv_decode_cascade_workspace_bytes(B, Hq, Hkv, D, MPB, MSB, max_group_size, bs,
+                                                        partition_tokens))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=query.device)
+    st = lib().pkv_paged_attention_decode_cascade(
+        _dev(query, "query"), _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache"),
+        _dev(prefix_tables, "prefix_tables"), MPB, _dev(prefix_lens, "prefix_lens"),
+        _dev(group_start, "group_start"), G, int(max_group_size), _dev(suffix_tables, "suffix_tables"),
+        MSB, _dev(suffix_lens, "suffix_lens"), B, Hq, Hkv, D, bs, NB, float(scale),
+        int(partition_tokens), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _dev(out, "out"), dt,
+        _stream_handle(stream, query.device))
+    _check(st, "pkv_paged_attention_decode_cascade")
     return out
 
 

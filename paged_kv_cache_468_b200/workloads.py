@@ -203,3 +203,27 @@ def make_decode_step(cfg: DecodeConfig, batch: Optional[int] = None,
 def kv_bytes(context_lens, num_kv_heads: int, head_dim: int, esize: int) -> int:
     """K+V bytes one decode step reads: every cached token row, for K and V."""
     return int(sum(int(x) for x in context_lens)) * num_kv_heads * head_dim * esize * 2
+
+
+def cascade_inputs(step: dict, prefix_tokens: int, samples: int) -> dict:
+    """Shared-prefix description of a step whose consecutive groups of
+    `samples` sequences share their first `prefix_tokens` tokens' blocks (as
+    make_decode_step builds them): one prefix table per group (the group's
+    first sequence's leading blocks) and each sequence's remaining blocks.
+    Only whole blocks are shared, so the prefix is rounded down to a block
+    multiple and the rest of a partly shared block stays in the suffix."""
+    bs = step["block_size"]
+    tables, lens = step["block_tables"], step["context_lens"]
+    B = tables.shape[0]
+    assert B % samples == 0
+    pb = prefix_tokens // bs
+    groups = B // samples
+    prefix_tables = tables[::samples, :max(pb, 1)].clone().contiguous()
+    prefix_lens = torch.full((groups,), pb * bs, dtype=torch.int32)
+    group_start = torch.arange(0, B + 1, samples, dtype=torch.int32)
+    msb = max(1, tables.shape[1] - pb)
+    suffix_tables = torch.full((B, msb), -1, dtype=torch.int32)
+    suffix_tables[:, :tables.shape[1] - pb] = tables[:, pb:]
+    suffix_lens = (lens - pb * bs).clamp(min=0).to(torch.int32)
+    return dict(prefix_tables=prefix_tables, prefix_lens=prefix_lens, group_start=group_start,
+                suffix_tables=suffix_tables, suffix_lens=suffix_lens, max_group_size=samples)

@@ -122,3 +122,18 @@ def test_binding_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         pkv.paged_attention_decode(q, kc, kc.clone(), torch.zeros(2, 4, dtype=torch.int32),
                                    torch.ones(2, dtype=torch.int32), 0.125)
+
+
+def test_cascade_workspace_and_validation():
+    L = pkv.lib()
+    # prefix records B*Hq*Pp and suffix records B*Hq*Ps, each (m, l, o[D]) floats
+    n = L.pkv_decode_cascade_workspace_bytes(256, 32, 8, 128, 125, 16, 8, 16, 0)
+    a = lambda x: (x + 255) // 256 * 256
+    rp, rs = 256 * 32 * 4, 256 * 32 * 1
+    exp = a(rp * 4); exp = a(exp + rp * 4); exp = a(exp + rp * 128 * 4)
+    exp = a(exp + rs * 4); exp = a(exp + rs * 4); exp = a(exp + rs * 128 * 4)
+    assert n == exp
+    assert L.pkv_decode_cascade_workspace_bytes(256, 32, 8, 128, 0, 16, 8, 16, 0) == 0
+    assert L.pkv_paged_attention_decode_cascade(None, None, None, None, 4, None, None, 1, 2, None, 4,
+                                                None, 2, 8, 8, 64, 16, 100, 1.0, 0, None, 0, None,
+                                                1, None) == pagedkv.ERR_INVALID_ARG

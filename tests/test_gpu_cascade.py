@@ -1,0 +1,128 @@
+"""Cascade (shared-prefix) decode on the GPU vs the fp64 oracle.
+
+The cascade computes exactly the decode over each sequence's full table
+(group prefix followed by its own blocks): the oracle runs the plain
+definition on the concatenated tables ("23.1 vLLM：高吞吐推理框架原理与部署",
+section 二.3: parallel samples share the prompt's blocks)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_468_b200 as pkv
+from paged_kv_cache_468_b200 import workloads
+from tests.parity_util import NTHREADS, TOL, max_abs_err, u16
+
+pytestmark = pytest.mark.gpu
+
+_DT = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+def _cascade_case(groups, prefix_blocks, suffix_tokens, Hq, Hkv, D, bs, dtype, seed):
+    """groups: sizes of consecutive groups (0-prefix groups allowed);
+    prefix_blocks[g]: shared blocks; suffix_tokens[b]: own tokens."""
+    g = torch.Generator().manual_seed(seed)
+    B = sum(groups)
+    sfx_blocks = [-(-t // bs) for t in suffix_tokens]
+    need = sum(prefix_blocks) + sum(sfx_blocks)
+    NB = need + 7
+    perm = torch.randperm(NB, generator=g).tolist()
+    cur = 0
+    prefix_tables = torch.full((len(groups), max(1, max(prefix_blocks))), -1, dtype=torch.int32)
+    for i, n in enumerate(prefix_blocks):
+        prefix_tables[i, :n] = torch.tensor(perm[cur:cur + n], dtype=torch.int32)
+        cur += n
+    msb = max(1, max(sfx_blocks))
+    suffix_tables = torch.full((B, msb), -1, dtype=torch.int32)
+    for b, n in enumerate(sfx_blocks):
+        suffix_tables[b, :n] = torch.tensor(perm[cur:cur + n], dtype=torch.int32)
+        cur += n
+    group_start = torch.tensor(np.concatenate([[0], np.cumsum(groups)]), dtype=torch.int32)
+    prefix_lens = torch.tensor([n * bs for n in prefix_blocks], dtype=torch.int32)
+    suffix_lens = torch.tensor(suffix_tokens, dtype=torch.int32)
+    # full tables for the oracle: prefix blocks, then own blocks
+    full_lens, rows = [], []
+    for gi, size in enumerate(groups):
+        for m in range(size):
+            b = int(group_start[gi]) + m
+            row = prefix_tables[gi, :prefix_blocks[gi]].tolist() + suffix_tables[b, :sfx_blocks[b]].tolist()
+            rows.append(row)
+            full_lens.append(prefix_blocks[gi] * bs + suffix_tokens[b])
+    mb = max(1, max(len(r) for r in rows))
+    full = torch.full((B, mb), -1, dtype=torch.int32)
+    for b, r in enumerate(rows):
+        if r:
+            full[b, :len(r)] = torch.tensor(r, dtype=torch.int32)
+    kc = torch.randn(NB, bs, Hkv, D, generator=g).to(_DT[dtype])
+    vc = torch.randn(NB, bs, Hkv, D, generator=g).to(_DT[dtype])
+    q = torch.randn(B, Hq, D, generator=g).to(_DT[dtype])
+    return dict(query=q, key_cache=kc, value_cache=vc, prefix_tables=prefix_tables,
+                prefix_lens=prefix_lens, group_start=group_start, suffix_tables=suffix_tables,
+                suffix_lens=suffix_lens, full_tables=full,
+                full_lens=torch.tensor(full_lens, dtype=torch.int32),
+                max_group_size=max(groups), scale=1.0 / np.sqrt(D), dtype=dtype)
+
+
+def _run(case, pt=0):
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in case.items()}
+    return pkv.paged_attention_decode_cascade(
+        d["query"], d["key_cache"], d["value_cache"], d["prefix_tables"], d["prefix_lens"],
+        d["group_start"], d["suffix_tables"], d["suffix_lens"], d["scale"],
+        max_group_size=d["max_group_size"], partition_tokens=pt)
+
+
+def _oracle(case):
+    return oracle.paged_attention_decode(u16(case["query"]), u16(case["key_cache"]),
+                                         u16(case["value_cache"]), case["full_tables"].numpy(),
+                                         case["full_lens"].numpy(), case["scale"], case["dtype"],
+                                         nthreads=NTHREADS)
+
+
+@pytest.fixture(autouse=True)
+def _clear_flags():
+    pkv.device_flags(clear=True)
+    yield
+    assert pkv.device_flags() == 0
+
+
+def test_cascade_full_shared_prefix_workload():
+    cfg = workloads.CONFIGS["shared_prefix"]
+    step = workloads.make_decode_step(cfg)
+    cas = workloads.cascade_inputs(step, cfg.shared_prefix, cfg.samples)
+    case = dict(query=step["query"], key_cache=step["key_cache"], value_cache=step["value_cache"],
+                full_tables=step["block_tables"], full_lens=step["context_lens"], scale=cfg.scale,
+                dtype=cfg.dtype, **cas)
+    ref = _oracle(case)
+    out = _run(case)
+    err, idx, finite = max_abs_err(out, ref)
+    assert finite and err <= TOL[cfg.dtype], (err, idx)
+    # and it agrees with the plain decode over the full tables
+    d = {k: v.cuda() for k, v in step.items() if isinstance(v, torch.Tensor)}
+    plain = pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"],
+                                       d["block_tables"], d["context_lens"], cfg.scale)
+    assert (plain.float() - out.float()).abs().max().item() <= TOL[cfg.dtype]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_cascade_irregular_groups(D, bs, dtype):
+    groups = [3, 1, 3]
+    prefix_blocks = [5, 0, 40]
+    suffix_tokens = [7, 0, 33, 100, 1, 16, 0]
+    case = _cascade_case(groups, prefix_blocks, suffix_tokens, 8, 2, D, bs, dtype, seed=D + bs)
+    ref = _oracle(case)
+    for pt in (0, 64):
+        err, idx, finite = max_abs_err(_run(case, pt), ref)
+        assert finite and err <= TOL[dtype], (pt, err, idx)
+
+
+@pytest.mark.parametrize("G,size", [(1, 8), (4, 8), (8, 16), (4, 32)])
+def test_cascade_group_shapes(G, size):
+    Hkv = 2
+    groups = [size, size]
+    case = _cascade_case(groups, [12, 20], list(range(1, 2 * size + 1)), G * Hkv, Hkv, 128, 16,
+                         "bf16", seed=G * 100 + size)
+    ref = _oracle(case)
+    err, idx, finite = max_abs_err(_run(case), ref)
+    assert finite and err <= TOL["bf16"], (err, idx)
