@@ -118,6 +118,31 @@ pkv_status pkv_kv_cache_write(const void *key, const void *value,
                               pkv_dtype dtype, void *stream);
 
 /*
+ * copy_blocks -- whole-block copies for copy-on-write and swapping ([FC] 二.3:
+ * a shared block is copied before a sequence writes into it; [YK] 三: the
+ * scheduler swaps a sequence's KV blocks out to CPU memory when the pool runs
+ * short and back in later).
+ *
+ *   src_key_cache, src_value_cache   [src_num_blocks, block_bytes]   read
+ *   dst_key_cache, dst_value_cache   [dst_num_blocks, block_bytes]   written
+ *   block_mapping                    [num_pairs][2] int32 (src, dst)  read
+ *
+ * Pair i copies source block block_mapping[i][0] to destination block
+ * block_mapping[i][1], K and V, bit for bit.  Caches and mapping are device
+ * memory or pinned host memory (reached through unified addressing), so the
+ * same call does copy-on-write inside one pool (source = destination caches),
+ * swap-out to host and swap-in.  block_bytes = block_size * num_kv_heads *
+ * head_dim * 2, a multiple of 16.  Destination blocks must be distinct and
+ * not also sources in the same call.  Out-of-range pairs are skipped and set
+ * PKV_DEVFLAG_BLOCK_RANGE.
+ */
+pkv_status pkv_copy_blocks(const void *src_key_cache, const void *src_value_cache,
+                           void *dst_key_cache, void *dst_value_cache,
+                           const int32_t *block_mapping, int num_pairs,
+                           int64_t src_num_blocks, int64_t dst_num_blocks, int64_t block_bytes,
+                           void *stream);
+
+/*
  * Partition plan of a decode call: the partition length in tokens the call
  * will use (a multiple of block_size) and the number of partitions per
  * sequence (1 = single pass, no workspace).  partition_tokens: > 0 requests
@@ -169,6 +194,36 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
                                       int partition_tokens, void *workspace,
                                       size_t workspace_bytes, void *out,
                                       pkv_dtype dtype, void *stream);
+
+/*
+ * paged_attention_prefill -- chunked prefill over the paged cache: each
+ * sequence brings a chunk of new query tokens whose K/V were already written
+ * through pkv_kv_cache_write ([MH] 2.1/3.3: the model runner's slot_mapping
+ * covers every token of the step; [YK] 三 for the block walk).
+ *
+ *   query          [num_tokens, num_heads, head_dim]                  device, read
+ *   query_start    [batch + 1] int32, ascending, <= num_tokens: sequence b's
+ *                  chunk is query rows query_start[b] .. query_start[b+1]-1
+ *                  (C_b tokens, C_b <= max_query_len)                 device, read
+ *   block_tables, context_lens (L_b >= C_b, the chunk included), caches as for
+ *                  pkv_paged_attention_decode
+ *   out            [T, num_heads, head_dim]                           device, written
+ *
+ * Query token i of sequence b sits at position L_b - C_b + i and attends
+ * causally over the sequence's tokens 0 .. L_b - C_b + i.  One CTA per tile of
+ * 64 (token, query head) rows of one sequence and kv head; a producer warp
+ * streams the blocks the tile needs into shared memory (TMA), eight consumer
+ * warps apply their rows to each block with mma.sync.  A chunk longer than
+ * its context or than max_query_len, or outside the query rows, sets
+ * PKV_DEVFLAG_CONTEXT_RANGE (such a chunk is clamped or skipped).
+ */
+pkv_status pkv_paged_attention_prefill(const void *query, int num_tokens, const int32_t *query_start,
+                                       int max_query_len, const void *key_cache,
+                                       const void *value_cache, const int32_t *block_tables,
+                                       int max_blocks, const int32_t *context_lens, int batch,
+                                       int num_heads, int num_kv_heads, int head_dim,
+                                       int block_size, int64_t num_blocks, float scale, void *out,
+                                       pkv_dtype dtype, void *stream);
 
 /*
  * paged_attention_decode_cascade -- decode for sequences that share a prefix

@@ -94,6 +94,11 @@ class Oracle:
         lib.pkvo_paged_attention_partitions.argtypes = [
             P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, dbl, i32, i32, i32,
             P, P, P, P]
+        lib.pkvo_paged_attention_prefill.restype = i32
+        lib.pkvo_paged_attention_prefill.argtypes = [
+            P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64, dbl, i32, P, P, i32]
+        lib.pkvo_copy_blocks.restype = i32
+        lib.pkvo_copy_blocks.argtypes = [P, P, P, i32, i64, i64, i64]
         lib.pkvo_lse_merge.restype = None
         lib.pkvo_lse_merge.argtypes = [P, P, P, i64, i32, i32, P]
         self.lib = lib
@@ -126,6 +131,40 @@ class Oracle:
                                           _ptr(key_cache), _ptr(value_cache), nb, block_size)
         if rc != OK:
             raise OracleError(rc, "kv_cache_write")
+
+    def paged_attention_prefill(self, query, query_start, key_cache, value_cache, block_tables,
+                                context_lens, scale: float, dtype: str,
+                                nthreads: int = 1) -> np.ndarray:
+        """Causal chunk attention: query [T, Hq, D] (uint16), query_start int32 [B+1]
+        -> unrounded fp64 [T, Hq, D]."""
+        q, kc, vc = _u16(query), _u16(key_cache), _u16(value_cache)
+        qs = _c(query_start, np.int32)
+        bt = _c(block_tables, np.int32)
+        cl = _c(context_lens, np.int32)
+        T, Hq, D = q.shape
+        nb, bs, Hkv, _ = kc.shape
+        mb = bt.shape[1]
+        out = np.zeros((T, Hq, D), dtype=np.float64)
+        scratch = np.empty(max(1, mb * bs) * nthreads, dtype=np.float64)
+        rc = self.lib.pkvo_paged_attention_prefill(
+            _ptr(q), _ptr(qs), _ptr(kc), _ptr(vc), _ptr(bt), mb, _ptr(cl), len(qs) - 1, Hq, Hkv,
+            D, bs, nb, float(scale), _DTYPE_CODE[dtype], _ptr(out), _ptr(scratch), nthreads)
+        if rc != OK:
+            raise OracleError(rc, "paged_attention_prefill")
+        return out
+
+    def copy_blocks(self, src_cache, dst_cache, mapping) -> None:
+        """In place: dst_cache[mapping[i, 1]] = src_cache[mapping[i, 0]] (bit copy)."""
+        src = _u16(src_cache)
+        if dst_cache.dtype != np.uint16 or not dst_cache.flags["C_CONTIGUOUS"]:
+            raise TypeError("dst_cache must be a C-contiguous uint16 array (written in place)")
+        mp = _c(mapping, np.int32).reshape(-1, 2)
+        elems = int(np.prod(src.shape[1:]))
+        assert int(np.prod(dst_cache.shape[1:])) == elems
+        rc = self.lib.pkvo_copy_blocks(_ptr(src), _ptr(dst_cache), _ptr(mp), mp.shape[0],
+                                       src.shape[0], dst_cache.shape[0], elems)
+        if rc != OK:
+            raise OracleError(rc, "copy_blocks")
 
     def paged_attention_decode(self, query, key_cache, value_cache, block_tables,
                                context_lens, scale: float, dtype: str,
@@ -209,3 +248,11 @@ def paged_attention_partitions(*a, **k):
 
 def lse_merge(*a, **k):
     return default().lse_merge(*a, **k)
+
+
+def copy_blocks(*a, **k):
+    return default().copy_blocks(*a, **k)
+
+
+def paged_attention_prefill(*a, **k):
+    return default().paged_attention_prefill(*a, **k)

@@ -137,6 +137,32 @@ int pkvo_kv_cache_write(const uint16_t *key, const uint16_t *value,
     return PKVO_OK;
 }
 
+/* ---- block copy: copy-on-write and swap ([FC] 二.3; [YK] 三 swap to CPU) -- */
+
+/*
+ * For every pair i: the whole block src_cache[mapping[2i]] (block_elems
+ * 16-bit elements) is copied bit for bit to dst_cache[mapping[2i+1]].  A
+ * block id outside its pool is an error: nothing is copied and
+ * PKVO_ERR_RANGE is returned.  Pairs are applied in order.
+ */
+int pkvo_copy_blocks(const uint16_t *src_cache, uint16_t *dst_cache, const int32_t *mapping,
+                     int num_pairs, int64_t src_blocks, int64_t dst_blocks, int64_t block_elems)
+{
+    if (num_pairs < 0 || block_elems <= 0)
+        return PKVO_ERR_ARG;
+    for (int i = 0; i < num_pairs; ++i)
+        if (mapping[2 * i] < 0 || mapping[2 * i] >= src_blocks || mapping[2 * i + 1] < 0 ||
+            mapping[2 * i + 1] >= dst_blocks)
+            return PKVO_ERR_RANGE;
+    for (int i = 0; i < num_pairs; ++i) {
+        const uint16_t *src = src_cache + (int64_t)mapping[2 * i] * block_elems;
+        uint16_t *dst = dst_cache + (int64_t)mapping[2 * i + 1] * block_elems;
+        for (int64_t e = 0; e < block_elems; ++e)
+            dst[e] = src[e];
+    }
+    return PKVO_OK;
+}
+
 /* ---- decode attention ([YK] 三, [FC] 二.2) ------------------------------ */
 
 static int check_tables(const int32_t *block_tables, int max_blocks,
@@ -158,21 +184,20 @@ static int check_tables(const int32_t *block_tables, int max_blocks,
 }
 
 /*
- * Attention of query head h of sequence b over that sequence's logical tokens
- * [j0, j1): writes the max score m, the softmax normaliser
+ * Attention of query row q (query head h) over a sequence's logical tokens
+ * [j0, j1), located through that sequence's block table: writes the max score m, the softmax normaliser
  * l = sum_j exp(s_j - m) and the normalised output o[d] = sum_j
  * exp(s_j - m) v_j[d] / l.  scores[] is caller scratch of j1-j0 entries;
  * it first holds the scores, then the weights.  An empty range gives m = -inf, l = 0, o = 0.
  */
-static void attend_range(const uint16_t *query, const uint16_t *key_cache,
+static void attend_range(const uint16_t *q, const uint16_t *key_cache,
                          const uint16_t *value_cache, const int32_t *table,
-                         int b, int h, int j0, int j1, int Hq, int Hkv, int D,
+                         int h, int j0, int j1, int Hq, int Hkv, int D,
                          int block_size, double scale, int dtype,
                          double *scores, double *m_out, double *l_out, double *o)
 {
     int group = Hq / Hkv;
     int kvh = h / group;
-    const uint16_t *q = query + ((int64_t)b * Hq + h) * D;
 
     for (int d = 0; d < D; ++d)
         o[d] = 0.0;
@@ -250,10 +275,62 @@ int pkvo_paged_attention_decode(const uint16_t *query, const uint16_t *key_cache
         double *sc = scratch;
 #endif
         double m, l;
-        attend_range(query, key_cache, value_cache,
-                     block_tables + (int64_t)b * max_blocks, b, h, 0,
+        attend_range(query + ((int64_t)b * Hq + h) * D, key_cache, value_cache,
+                     block_tables + (int64_t)b * max_blocks, h, 0,
                      context_lens[b], Hq, Hkv, D, block_size, scale, dtype, sc,
                      &m, &l, out + bh * D);
+    }
+    return PKVO_OK;
+}
+
+/*
+ * Chunked prefill: sequence b has query_start[b+1] - query_start[b] = C_b new
+ * query tokens, the last C_b of its context_lens[b] = L_b cached tokens (their
+ * K/V already written).  Query token i of b sits at logical position
+ * p = L_b - C_b + i and attends over the cached tokens 0 .. p (causal):
+ *   out[query_start[b] + i, h, :] = softmax_j<=p(scale * <q, K_j>) . V_j
+ * query and out are [total_tokens, Hq, D].  Returns PKVO_ERR_RANGE if a
+ * chunk is longer than its context or a context does not fit the table.
+ */
+int pkvo_paged_attention_prefill(const uint16_t *query, const int32_t *query_start,
+                                 const uint16_t *key_cache, const uint16_t *value_cache,
+                                 const int32_t *block_tables, int max_blocks,
+                                 const int32_t *context_lens, int batch, int Hq, int Hkv, int D,
+                                 int block_size, int64_t num_blocks, double scale, int dtype,
+                                 double *out, double *scratch, int nthreads)
+{
+    if (batch < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || D <= 0 ||
+        block_size <= 0 || max_blocks <= 0 || nthreads <= 0)
+        return PKVO_ERR_ARG;
+    int rc = check_tables(block_tables, max_blocks, context_lens, batch, block_size, num_blocks);
+    if (rc != PKVO_OK)
+        return rc;
+    for (int b = 0; b < batch; ++b) {
+        int C = query_start[b + 1] - query_start[b];
+        if (C < 0 || C > context_lens[b])
+            return PKVO_ERR_RANGE;
+    }
+    int64_t span = (int64_t)max_blocks * block_size;
+    int64_t rows = (int64_t)query_start[batch] * Hq;
+#pragma omp parallel for schedule(dynamic, 16) num_threads(nthreads)
+    for (int64_t th = 0; th < rows; ++th) {
+        int64_t t = th / Hq;
+        int h = (int)(th % Hq);
+        int b = 0;
+        while (query_start[b + 1] <= t)     /* the sequence that owns token t */
+            ++b;
+        int i = (int)(t - query_start[b]);
+        int C = query_start[b + 1] - query_start[b];
+        int p = context_lens[b] - C + i;
+#ifdef _OPENMP
+        double *sc = scratch + span * omp_get_thread_num();
+#else
+        double *sc = scratch;
+#endif
+        double m, l;
+        attend_range(query + th * D, key_cache, value_cache,
+                     block_tables + (int64_t)b * max_blocks, h, 0, p + 1, Hq, Hkv, D,
+                     block_size, scale, dtype, sc, &m, &l, out + th * D);
     }
     return PKVO_OK;
 }
@@ -290,8 +367,8 @@ int pkvo_paged_attention_partitions(const uint16_t *query, const uint16_t *key_c
                 int j1 = j0 + partition_tokens;
                 if (j1 > L)
                     j1 = L;
-                attend_range(query, key_cache, value_cache,
-                             block_tables + (int64_t)b * max_blocks, b, h, j0, j1,
+                attend_range(query + ((int64_t)b * Hq + h) * D, key_cache, value_cache,
+                             block_tables + (int64_t)b * max_blocks, h, j0, j1,
                              Hq, Hkv, D, block_size, scale, dtype, scratch,
                              &m_out[idx], &l_out[idx], o_out + idx * D);
             }

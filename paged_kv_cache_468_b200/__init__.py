@@ -11,6 +11,7 @@ from .pagedkv import (  # noqa: F401
     F16,
     BlockAllocator,
     PagedKVError,
+    copy_blocks,
     decode_plan,
     decode_workspace_bytes,
     device_flags,
@@ -18,6 +19,7 @@ from .pagedkv import (  # noqa: F401
     lib,
     paged_attention_decode,
     paged_attention_decode_cascade,
+    paged_attention_prefill,
     selftest_bounded_wait,
     version,
 )

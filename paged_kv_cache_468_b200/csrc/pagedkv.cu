@@ -292,6 +292,41 @@ pkv_status pkv_device_flags(int device, unsigned int *flags, int clear)
     return st;
 }
 
+pkv_status pkv_copy_blocks(const void *src_key_cache, const void *src_value_cache,
+                           void *dst_key_cache, void *dst_value_cache, const int32_t *block_mapping,
+                           int num_pairs, int64_t src_num_blocks, int64_t dst_num_blocks,
+                           int64_t block_bytes, void *stream)
+{
+    if (num_pairs < 0 || src_num_blocks <= 0 || dst_num_blocks <= 0 || block_bytes <= 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_pairs=%d src_num_blocks=%lld dst_num_blocks=%lld "
+                    "block_bytes=%lld", num_pairs, (long long)src_num_blocks,
+                    (long long)dst_num_blocks, (long long)block_bytes);
+    if (block_bytes % 16 != 0)
+        return fail(PKV_ERR_UNSUPPORTED, "block_bytes %lld is not a multiple of 16",
+                    (long long)block_bytes);
+    if (num_pairs == 0)
+        return PKV_OK;
+    if (!src_key_cache || !src_value_cache || !dst_key_cache || !dst_value_cache || !block_mapping)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(src_key_cache) || !aligned16(src_value_cache) || !aligned16(dst_key_cache) ||
+        !aligned16(dst_value_cache))
+        return fail(PKV_ERR_MISALIGNED, "cache pointers must be 16-byte aligned");
+    if (reinterpret_cast<uintptr_t>(block_mapping) & 7u)
+        return fail(PKV_ERR_MISALIGNED, "block_mapping must be 8-byte aligned");
+    const int64_t vec_per_block = block_bytes / 16;
+    const int64_t n = (int64_t)num_pairs * 2 * vec_per_block;
+    const int threads = 256;
+    const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 16);
+    pkv::copy_blocks_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(src_key_cache), static_cast<const uint4 *>(src_value_cache),
+        static_cast<uint4 *>(dst_key_cache), static_cast<uint4 *>(dst_value_cache), block_mapping,
+        num_pairs, src_num_blocks, dst_num_blocks, vec_per_block);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return cuda_fail(e, "copy_blocks_kernel launch");
+    return PKV_OK;
+}
+
 pkv_status pkv_selftest_bounded_wait(int64_t limit_ns, void *stream)
 {
     if (limit_ns <= 0 || limit_ns > 10000000000ll)
@@ -662,6 +697,101 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
                            : go(pkv::lse_merge_cascade_kernel<false, 128, NT>, 128);
     if (e != cudaSuccess)
         return cuda_fail(e, "lse_merge_cascade_kernel launch");
+    return PKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Chunked prefill
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kPrefillWarps = 8;   // consumer warps: 64 query rows per CTA
+
+template <int D, int BS, bool BF16>
+cudaError_t launch_prefill(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::PrefillArgs &p,
+                           int max_query_len, cudaStream_t st)
+{
+    constexpr int NWQ = kPrefillWarps;
+    constexpr int S = BS == 16 ? 4 : 3;
+    using Shape = pkv::DecodeShape<D, BS, 1, S>;
+    constexpr int smem = S * Shape::kStageBytes + 1024;
+    auto kern = pkv::prefill_kernel<D, BS, BF16, NWQ, S>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess)
+        return e;
+    const int64_t rows = (int64_t)max_query_len * p.group;
+    const dim3 grid((unsigned)((rows + NWQ * 8 - 1) / (NWQ * 8)), (unsigned)p.num_kv_heads,
+                    (unsigned)p.batch);
+    return launch_pdl(kern, grid, dim3((NWQ + 1) * 32), smem, st, mk, mv, p);
+}
+
+template <bool BF16>
+cudaError_t dispatch_prefill(int D, int bs, const CUtensorMap &mk, const CUtensorMap &mv,
+                             const pkv::PrefillArgs &p, int max_query_len, cudaStream_t st)
+{
+    if (D == 64 && bs == 16) return launch_prefill<64, 16, BF16>(mk, mv, p, max_query_len, st);
+    if (D == 64 && bs == 32) return launch_prefill<64, 32, BF16>(mk, mv, p, max_query_len, st);
+    if (D == 128 && bs == 16) return launch_prefill<128, 16, BF16>(mk, mv, p, max_query_len, st);
+    return launch_prefill<128, 32, BF16>(mk, mv, p, max_query_len, st);
+}
+
+}  // namespace
+
+extern "C" pkv_status pkv_paged_attention_prefill(
+    const void *query, int num_tokens, const int32_t *query_start, int max_query_len,
+    const void *key_cache,
+    const void *value_cache, const int32_t *block_tables, int max_blocks,
+    const int32_t *context_lens, int batch, int num_heads, int num_kv_heads, int head_dim,
+    int block_size, int64_t num_blocks, float scale, void *out, pkv_dtype dtype, void *stream)
+{
+    pkv_status s = check_shapes(batch, num_heads, num_kv_heads, head_dim, max_blocks, block_size);
+    if (s != PKV_OK)
+        return s;
+    if (dtype != PKV_F16 && dtype != PKV_BF16)
+        return fail(PKV_ERR_INVALID_ARG, "dtype %d", (int)dtype);
+    if (num_tokens < 0)
+        return fail(PKV_ERR_INVALID_ARG, "num_tokens %d", num_tokens);
+    if (max_query_len < 0 || max_query_len > max_blocks * block_size)
+        return fail(PKV_ERR_INVALID_ARG, "max_query_len %d (0 .. max_blocks*block_size)", max_query_len);
+    if ((int64_t)max_query_len * (num_heads / num_kv_heads) > ((int64_t)1 << 30))
+        return fail(PKV_ERR_UNSUPPORTED, "max_query_len too large");
+    if (num_blocks <= 0 || num_blocks * block_size >= ((int64_t)1 << 31))
+        return fail(PKV_ERR_INVALID_ARG, "num_blocks %lld: need 0 < num_blocks*block_size < 2^31",
+                    (long long)num_blocks);
+    if (!std::isfinite(scale))
+        return fail(PKV_ERR_INVALID_ARG, "scale is not finite");
+    if (batch == 0 || max_query_len == 0 || num_tokens == 0)
+        return PKV_OK;
+    if (!query || !query_start || !key_cache || !value_cache || !block_tables || !context_lens || !out)
+        return fail(PKV_ERR_INVALID_ARG, "null pointer");
+    if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
+        return fail(PKV_ERR_MISALIGNED, "query/cache/out pointers must be 16-byte aligned");
+    CUtensorMap mk, mv;
+    if ((s = make_cache_map(&mk, key_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
+        return s;
+    if ((s = make_cache_map(&mv, value_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
+        return s;
+    pkv::PrefillArgs p;
+    p.query = static_cast<const uint16_t *>(query);
+    p.query_start = query_start;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    p.out = static_cast<uint16_t *>(out);
+    p.batch = batch;
+    p.num_tokens = num_tokens;
+    p.max_query_len = max_query_len;
+    p.max_blocks = max_blocks;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_heads / num_kv_heads;
+    p.num_blocks = (int)num_blocks;
+    p.scale_log2 = (float)((double)scale * 1.4426950408889634);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e = dtype == PKV_BF16
+                        ? dispatch_prefill<true>(head_dim, block_size, mk, mv, p, max_query_len, st)
+                        : dispatch_prefill<false>(head_dim, block_size, mk, mv, p, max_query_len, st);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "prefill_kernel launch");
     return PKV_OK;
 }
 

@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_version.argtypes = []
         L.pkv_device_flags.restype = i32
         L.pkv_device_flags.argtypes = [i32, ctypes.POINTER(ctypes.c_uint), i32]
+        L.pkv_copy_blocks.restype = i32
+        L.pkv_copy_blocks.argtypes = [P, P, P, P, P, i32, i64, i64, i64, P]
         L.pkv_selftest_bounded_wait.restype = i32
         L.pkv_selftest_bounded_wait.argtypes = [i64, P]
         L.pkv_kv_cache_write.restype = i32
@@ -67,6 +69,9 @@ def lib() -> ctypes.CDLL:
         L.pkv_paged_attention_decode.restype = i32
         L.pkv_paged_attention_decode.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, i64,
                                                  f32, i32, P, sz, P, i32, P]
+        L.pkv_paged_attention_prefill.restype = i32
+        L.pkv_paged_attention_prefill.argtypes = [P, i32, P, i32, P, P, P, i32, P, i32, i32, i32,
+                                                  i32, i32, i64, f32, P, i32, P]
         L.pkv_decode_cascade_workspace_bytes.restype = sz
         L.pkv_decode_cascade_workspace_bytes.argtypes = [i32] * 9
         L.pkv_paged_attention_decode_cascade.restype = i32
@@ -133,6 +138,36 @@ def device_flags(device: Optional[int] = None, clear: bool = True) -> int:
     v = ctypes.c_uint(0)
     _check(lib().pkv_device_flags(dev, ctypes.byref(v), int(clear)), "pkv_device_flags")
     return v.value
+
+
+def _block_ptr(t: torch.Tensor, name: str) -> int:
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be a CUDA tensor or pinned host memory")
+    return t.data_ptr()
+
+
+def copy_blocks(src_key_cache: torch.Tensor, src_value_cache: torch.Tensor,
+                dst_key_cache: torch.Tensor, dst_value_cache: torch.Tensor,
+                block_mapping: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """dst[block_mapping[i, 1]] = src[block_mapping[i, 0]] for K and V (copy-on-write
+    within one pool, or swap between a device pool and pinned host memory)."""
+    if block_mapping.dtype != torch.int32 or block_mapping.dim() != 2 or block_mapping.shape[1] != 2:
+        raise ValueError("block_mapping must be int32 [num_pairs, 2]")
+    for t in (src_value_cache, dst_key_cache, dst_value_cache):
+        if t.shape[1:] != src_key_cache.shape[1:] or t.dtype != src_key_cache.dtype:
+            raise ValueError("all caches must share block shape and element type")
+    if src_value_cache.shape[0] != src_key_cache.shape[0] or dst_value_cache.shape[0] != dst_key_cache.shape[0]:
+        raise ValueError("K and V pools must have the same number of blocks")
+    block_bytes = src_key_cache[0].numel() * src_key_cache.element_size()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    st = lib().pkv_copy_blocks(
+        _block_ptr(src_key_cache, "src_key_cache"), _block_ptr(src_value_cache, "src_value_cache"),
+        _block_ptr(dst_key_cache, "dst_key_cache"), _block_ptr(dst_value_cache, "dst_value_cache"),
+        _block_ptr(block_mapping, "block_mapping"), block_mapping.shape[0], src_key_cache.shape[0],
+        dst_key_cache.shape[0], block_bytes, _stream_handle(stream, dev))
+    _check(st, "pkv_copy_blocks")
 
 
 def selftest_bounded_wait(limit_ns: int, stream: Optional[torch.cuda.Stream] = None) -> None:
@@ -225,6 +260,33 @@ def paged_attention_decode(query: torch.Tensor, key_cache: torch.Tensor, value_c
         bs, NB, float(scale), int(partition_tokens), ws_ptr, ws_bytes, _dev(out, "out"), dt,
         _stream_handle(stream, query.device))
     _check(st, "pkv_paged_attention_decode")
+    return out
+
+
+def paged_attention_prefill(query: torch.Tensor, query_start: torch.Tensor, max_query_len: int,
+                            key_cache: torch.Tensor, value_cache: torch.Tensor,
+                            block_tables: torch.Tensor, context_lens: torch.Tensor, scale: float,
+                            out: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Causal chunk attention: query [T, Hq, D], query_start int32 [B+1] -> out [T, Hq, D]."""
+    if query.dim() != 3:
+        raise ValueError("query must be [total_tokens, num_heads, head_dim]")
+    T, Hq, D = query.shape
+    NB, bs, Hkv, _ = key_cache.shape
+    B = block_tables.shape[0]
+    if query_start.dtype != torch.int32 or query_start.shape != (B + 1,):
+        raise ValueError("query_start must be int32 [batch + 1]")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise ValueError("block_tables / context_lens must be int32")
+    dt = _dtype_code(query)
+    if out is None:
+        out = torch.empty_like(query)
+    st = lib().pkv_paged_attention_prefill(
+        _dev(query, "query"), T, _dev(query_start, "query_start"), int(max_query_len),
+        _dev(key_cache, "key_cache"), _dev(value_cache, "value_cache"),
+        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"),
+        B, Hq, Hkv, D, bs, NB, float(scale), _dev(out, "out"), dt, _stream_handle(stream, query.device))
+    _check(st, "pkv_paged_attention_prefill")
     return out
 
 

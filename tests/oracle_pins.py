@@ -351,4 +351,68 @@ def pin_write_roundtrip(orc):
     assert np.array_equal(out[0], ref)
 
 
+def pin_copy_blocks(orc):
+    """Copied blocks equal their sources bit for bit; other blocks untouched;
+    a copy-on-write then a one-token decode reads the source's values."""
+    import oracle
+    rng = np.random.default_rng(17)
+    NB, bs, Hkv, D = 9, 4, 2, 8
+    src = codes(rng.standard_normal((NB, bs, Hkv, D)), "bf16")
+    dst = codes(rng.standard_normal((5, bs, Hkv, D)), "bf16")
+    before = dst.copy()
+    mapping = np.array([[7, 0], [2, 3], [7, 4]], np.int32)
+    orc.copy_blocks(src, dst, mapping)
+    for s_, d_ in mapping:
+        assert np.array_equal(dst[d_], src[s_])
+    assert np.array_equal(dst[[1, 2]], before[[1, 2]])
+    try:
+        orc.copy_blocks(src, dst, np.array([[0, 5]], np.int32))     # dst out of range
+        raise AssertionError("out-of-range block accepted")
+    except oracle.OracleError as e:
+        assert e.code == oracle.ERR_RANGE
+    # copy-on-write inside one pool, then decode block 1 as a one-token context
+    pool = codes(rng.standard_normal((4, bs, Hkv, D)), "f16")
+    orc.copy_blocks(pool.copy(), pool, np.array([[3, 1]], np.int32))
+    q = codes(rng.standard_normal((1, Hkv, D)), "f16")
+    out = orc.paged_attention_decode(q, pool, pool, np.array([[1]], np.int32),
+                                     np.array([1], np.int32), 0.5, "f16")
+    assert np.array_equal(out[0], values(pool[3, 0], "f16").numpy())
+
+
+def pin_prefill_causal_sdpa(orc):
+    """Chunked prefill equals torch SDPA with an explicit causal mask on the dense
+    layout (query token i of a C-token chunk at position L-C+i sees keys 0..L-C+i),
+    and a chunk's last token equals the decode of the whole context."""
+    cases = [(3, 4, 2, 16, 4, [9, 20, 5], [3, 20, 1], "bf16"),
+             (2, 8, 8, 8, 16, [33, 17], [16, 5], "f16")]
+    for ci, (B, Hq, Hkv, D, bs, lens, chunks, dt) in enumerate(cases):
+        case = dense_case(B, Hq, Hkv, D, bs, lens, dt, seed=200 + ci)
+        rng = np.random.default_rng(300 + ci)
+        T = sum(chunks)
+        qf = rng.standard_normal((T, Hq, D)).astype(np.float32)
+        q = codes(qf, dt)
+        qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+        scale = 1.0 / math.sqrt(D)
+        got = orc.paged_attention_prefill(q, qs, case["kc"], case["vc"], case["table"],
+                                          case["lens"], scale, dt)
+        qv = values(q, dt)
+        for b in range(B):
+            L, C = lens[b], chunks[b]
+            k = values(case["dense_k"][b], dt)[:L].permute(1, 0, 2)     # [Hkv, L, D]
+            v = values(case["dense_v"][b], dt)[:L].permute(1, 0, 2)
+            k = k.repeat_interleave(Hq // Hkv, 0)
+            v = v.repeat_interleave(Hq // Hkv, 0)
+            qb = qv[qs[b]:qs[b + 1]].permute(1, 0, 2)                   # [Hq, C, D]
+            pos = torch.arange(L - C, L)[:, None]
+            mask = torch.arange(L)[None, :] <= pos                      # [C, L]
+            ref = F.scaled_dot_product_attention(qb, k, v, attn_mask=mask, scale=scale)
+            err = np.abs(got[qs[b]:qs[b + 1]] - ref.permute(1, 0, 2).numpy()).max()
+            assert err < 1e-12, (ci, b, err)
+            # last chunk token == decode of the full context with that query
+            dec = orc.paged_attention_decode(q[qs[b + 1] - 1][None], case["kc"], case["vc"],
+                                             case["table"][b:b + 1], case["lens"][b:b + 1],
+                                             scale, dt)
+            assert np.array_equal(dec[0], got[qs[b + 1] - 1])
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

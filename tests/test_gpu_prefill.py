@@ -1,0 +1,73 @@
+"""Chunked prefill on the GPU vs the fp64 oracle (causal attention of each
+chunk token over its sequence's paged cache)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_468_b200 as pkv
+from tests.parity_util import NTHREADS, TOL, custom, max_abs_err, u16
+
+pytestmark = pytest.mark.gpu
+
+_DT = {"f16": torch.float16, "bf16": torch.bfloat16}
+
+
+@pytest.fixture(autouse=True)
+def _clear_flags():
+    pkv.device_flags(clear=True)
+    yield
+    assert pkv.device_flags() == 0
+
+
+def _case(lens, chunks, Hq, Hkv, D, bs, dtype, seed):
+    step = custom("pf", len(lens), Hq, Hkv, D, bs, dtype, lens, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    T = sum(chunks)
+    q = torch.randn(T, Hq, D, generator=g).to(_DT[dtype])
+    qs = torch.tensor(np.concatenate([[0], np.cumsum(chunks)]), dtype=torch.int32)
+    return step, q, qs
+
+
+def _check(step, q, qs, chunks):
+    ref = oracle.paged_attention_prefill(u16(q), qs.numpy(), u16(step["key_cache"]),
+                                         u16(step["value_cache"]), step["block_tables"].numpy(),
+                                         step["context_lens"].numpy(), step["scale"],
+                                         step["dtype"], nthreads=NTHREADS)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
+    out = pkv.paged_attention_prefill(q.cuda(), qs.cuda(), max(chunks), d["key_cache"],
+                                      d["value_cache"], d["block_tables"], d["context_lens"],
+                                      step["scale"])
+    err, idx, finite = max_abs_err(out, ref)
+    assert finite and err <= TOL[step["dtype"]], (err, idx)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("bs", [16, 32])
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_prefill_ragged_chunks(D, bs, dtype):
+    lens = [1, 17, 100, 300, 33, 64]
+    chunks = [1, 17, 37, 300, 5, 1]          # whole contexts, partial chunks, single tokens
+    step, q, qs = _case(lens, chunks, 8, 2, D, bs, dtype, seed=D + bs)
+    _check(step, q, qs, chunks)
+
+
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_prefill_group_sizes(G):
+    lens = [700, 129, 520]
+    chunks = [512, 129, 7]
+    step, q, qs = _case(lens, chunks, 4 * G, 4, 128, 16, "bf16", seed=G)
+    _check(step, q, qs, chunks)
+
+
+def test_prefill_last_token_equals_decode():
+    lens, chunks = [200, 61], [40, 61]
+    step, q, qs = _case(lens, chunks, 8, 2, 128, 16, "bf16", seed=77)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
+    out = pkv.paged_attention_prefill(q.cuda(), qs.cuda(), max(chunks), d["key_cache"],
+                                      d["value_cache"], d["block_tables"], d["context_lens"],
+                                      step["scale"])
+    last = q[qs[1:] - 1].cuda()                          # each chunk's last token
+    dec = pkv.paged_attention_decode(last, d["key_cache"], d["value_cache"], d["block_tables"],
+                                     d["context_lens"], step["scale"], partition_tokens=-1)
+    assert (out[qs[1:].long().cuda() - 1].float() - dec.float()).abs().max().item() <= TOL["bf16"]

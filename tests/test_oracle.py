@@ -36,6 +36,11 @@ MUTANTS = {
     "write_skips_slot_zero": ("if (slot < 0)\n            continue;", "if (slot <= 0)\n            continue;"),
     "write_value_from_key": ("value_cache[dst + d] = value[src + d];", "value_cache[dst + d] = key[src + d];"),
     "merge_drops_partition_sum": ("double w = exp(mr[p] - M) * lr[p];", "double w = exp(mr[p] - M);"),
+    "copy_uses_dst_index_for_src": ("const uint16_t *src = src_cache + (int64_t)mapping[2 * i] * block_elems;",
+                                    "const uint16_t *src = src_cache + (int64_t)mapping[2 * i + 1] * block_elems;"),
+    "prefill_not_causal": ("                     block_tables + (int64_t)b * max_blocks, h, 0, p + 1, Hq, Hkv, D,",
+                           "                     block_tables + (int64_t)b * max_blocks, h, 0, context_lens[b], Hq, Hkv, D,"),
+    "prefill_off_by_one": ("int p = context_lens[b] - C + i;", "int p = context_lens[b] - C + i - 1;"),
     "merge_sign_flipped": ("double w = exp(mr[p] - M) * lr[p];", "double w = exp(M - mr[p]) * lr[p];"),
 }
 
