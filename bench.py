@@ -29,6 +29,7 @@ import sys
 import threading
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -354,6 +355,23 @@ def run_gpu(args, cfg, world, rank, local):
         one_step()
     torch.cuda.synchronize()
 
+    # optional: the step as a CUDA graph (same kernels, no per-launch host work)
+    step_fn = one_step
+    graph_note = "off"
+    if args.graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                one_step()
+            for _ in range(3):
+                graph.replay()
+            torch.cuda.synchronize()
+            step_fn = graph.replay
+            graph_note = "on"
+        except Exception as exc:   # capture unsupported here: plain launches
+            graph_note = f"capture failed ({type(exc).__name__}); plain launches"
+            torch.cuda.synchronize()
+
     # ---- device-timed region (inputs resident in HBM): K whole steps ----
     K = args.steps
     sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
@@ -367,7 +385,7 @@ def run_gpu(args, cfg, world, rank, local):
         sampler.mark(True)
     t_start.record(stream)
     for _ in range(K):
-        one_step()
+        step_fn()
     t_end.record(stream)
     torch.cuda.synchronize()
     if sampler:
@@ -468,7 +486,7 @@ def run_gpu(args, cfg, world, rank, local):
                        "num_blocks": NB, "max_blocks": MB,
                        "context_tokens": nbytes["kv_tokens"],
                        "partition_tokens": plan_pt, "num_partitions": plan_np,
-                       "cascade": cascade,
+                       "cascade": cascade, "cuda_graph": graph_note,
                        "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                        "l2": (f"inputs larger than L2: {nbytes['kv_unique'] / 1e6:.0f} MB of K/V "
                               f"per step vs 126 MB L2, no flush")
@@ -489,6 +507,94 @@ def run_gpu(args, cfg, world, rank, local):
     return 0
 
 
+def _time_loop(fn, steps, warmup, stream):
+    """Mean ms per call of fn over `steps` calls (CUDA events on `stream`)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps
+
+
+def run_other_op(args, cfg, world, rank, local):
+    """The NEXT-row operations, one GPU: chunked prefill (tensor roofline),
+    copy-on-write block copies (HBM roofline) and swap-out to pinned host."""
+    import paged_kv_cache_468_b200 as pkv
+
+    dev = torch.device("cuda", local)
+    step = workloads.make_decode_step(cfg)
+    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
+    B, Hq, D = d["query"].shape
+    NB, bs, Hkv, _ = d["key_cache"].shape
+    stream = torch.cuda.current_stream(dev)
+    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) \
+        if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    line = {"impl": "pagedkv", "op": args.op, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "dtype": cfg.dtype, "data": "synthetic",
+            "config": {"workload": cfg.name, "description": cfg.description}}
+    if args.op == "prefill":
+        lens = [int(x) for x in step["context_lens"]]
+        chunks = [min(args.chunk, L) for L in lens]
+        g = torch.Generator().manual_seed(cfg.seed + 7)
+        T = sum(chunks)
+        q = torch.randn(T, Hq, D, generator=g).to(step["query"].dtype).to(dev)
+        qs = torch.tensor([0] + list(np.cumsum(chunks)), dtype=torch.int32, device=dev)
+        out = torch.empty_like(q)
+        fn = lambda: pkv.paged_attention_prefill(q, qs, max(chunks), d["key_cache"], d["value_cache"],
+                                                 d["block_tables"], d["context_lens"], d["scale"],
+                                                 out=out)
+        ms = _time_loop(fn, args.steps, args.warmup, stream)
+        # causal attention FLOPs: QK and PV, 2 flops per MAC, over keys 0..p
+        keys = sum(sum(L - C + i + 1 for i in range(C)) for L, C in zip(lens, chunks))
+        flops = 4.0 * D * Hq * keys
+        peak = float(peaks.get("bf16_tflops", 1590.0))
+        line.update(metric="chunked prefill attention TFLOP/s", unit="TFLOP/s",
+                    value=round(flops / (ms * 1e-3) / 1e12, 2), ms_per_step=round(ms, 4),
+                    higher_is_better=True, tokens_per_s=round(T / (ms * 1e-3), 1),
+                    roofline={"bound": "tensor", "achieved": round(flops / (ms * 1e-3) / 1e12, 2),
+                              "peak": peak, "unit": "TFLOP/s",
+                              "frac": round(flops / (ms * 1e-3) / 1e12 / peak, 4),
+                              "peak_source": "MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16)",
+                              "note": "mma.sync m16n8k16 (legacy tensor path)"})
+        line["config"].update(chunk=args.chunk, query_tokens=T)
+    else:
+        n = min(args.pairs, NB // 2)
+        g = torch.Generator().manual_seed(cfg.seed + 11)
+        perm = torch.randperm(NB, generator=g)
+        mapping = torch.stack([perm[:n], perm[n:2 * n]], 1).to(torch.int32).to(dev)
+        block_bytes = bs * Hkv * D * 2
+        if args.op == "copy":
+            fn = lambda: pkv.copy_blocks(d["key_cache"], d["value_cache"], d["key_cache"],
+                                         d["value_cache"], mapping)
+            moved = 2 * 2 * n * block_bytes                    # K and V, read + write
+            peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+            bound = "hbm"
+        else:
+            hk = torch.empty((n,) + tuple(d["key_cache"].shape[1:]), dtype=d["key_cache"].dtype).pin_memory()
+            hv = torch.empty_like(hk).pin_memory()
+            out_map = torch.stack([perm[:n], torch.arange(n)], 1).to(torch.int32).to(dev)
+            fn = lambda: pkv.copy_blocks(d["key_cache"], d["value_cache"], hk, hv, out_map)
+            moved = 2 * n * block_bytes                        # bytes that cross to the host
+            peak = None
+            bound = "host link"
+        ms = _time_loop(fn, args.steps, args.warmup, stream)
+        gbs = moved / (ms * 1e-3) / 1e9
+        line.update(metric=f"block {args.op} GB/s", unit="GB/s", value=round(gbs, 2),
+                    ms_per_step=round(ms, 4), higher_is_better=True,
+                    roofline={"bound": bound, "achieved": round(gbs, 2), "peak": peak,
+                              "unit": "GB/s", "frac": round(gbs / peak, 4) if peak else None})
+        line["config"].update(pairs=n, block_bytes=block_bytes)
+    line["device_flags"] = pkv.device_flags(clear=True)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def dataclass_replace(cfg, **kw):
     import dataclasses
     return dataclasses.replace(cfg, **kw)
@@ -501,6 +607,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--config", default=workloads.HEADLINE, choices=sorted(workloads.CONFIGS))
     ap.add_argument("--impl", default="pagedkv", choices=["pagedkv", "reference"])
+    ap.add_argument("--op", default="decode", choices=["decode", "prefill", "copy", "swap"],
+                    help="decode step (the contract line) or a NEXT-row operation")
+    ap.add_argument("--chunk", type=int, default=512, help="prefill chunk tokens per sequence")
+    ap.add_argument("--pairs", type=int, default=2048, help="block pairs for --op copy/swap")
     ap.add_argument("--partition-tokens", type=int, default=None,
                     help="override the workload's partition request (0 auto, <0 never)")
     ap.add_argument("--e2e-steps", type=int, default=200)
@@ -509,6 +619,8 @@ def main(argv=None):
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--cascade", default="auto", choices=["auto", "on", "off"],
                     help="shared-prefix decode (auto: for workloads with a shared prefix)")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay the step as a CUDA graph in the timed loop")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true")
@@ -526,6 +638,8 @@ def main(argv=None):
     if world != args.gpus and rank == 0:
         print(f"note: --gpus {args.gpus} but WORLD_SIZE {world}; using {world}", file=sys.stderr)
     try:
+        if args.op != "decode":
+            return run_other_op(args, cfg, world, rank, local)
         return run_gpu(args, cfg, world, rank, local)
     finally:
         if world > 1:
