@@ -340,6 +340,40 @@ pkv_status pkv_alloc_append(pkv_alloc *a, int32_t *blocks, int capacity, int *n,
  * outside the pool or already free. */
 pkv_status pkv_alloc_free(pkv_alloc *a, const int32_t *blocks, int n);
 
+/* ---- automatic prefix caching ([FC] 五.4; [MH] 2.3) --------------------
+ *
+ * Full blocks can be registered under a hash of their tokens chained with
+ * the previous block's hash, so a new request whose prompt starts with the
+ * same tokens reuses those blocks (and skips recomputing their K/V).  A
+ * registered block whose reference count drops to zero stays findable: it
+ * is "evictable" and is reused by a later lookup, or given out (and
+ * forgotten) by new_seq / append only when the free list is empty, least
+ * recently released first.  pkv_alloc_num_free counts free and evictable
+ * blocks.
+ */
+
+/* Hash of a block's n tokens chained to the previous block's hash (0 for the
+ * first block); never returns 0. */
+uint64_t pkv_block_hash(uint64_t parent_hash, const int32_t *tokens, int n);
+
+/* Register an in-use block (refcount > 0) under `hash`.  No-op if the block
+ * is already registered or another block holds that hash. */
+pkv_status pkv_alloc_cache_insert(pkv_alloc *a, uint64_t hash, int32_t block);
+
+/* Block registered under `hash` with its refcount raised by one (a released
+ * block is revived), or -1 if none. */
+int32_t pkv_alloc_cache_lookup(pkv_alloc *a, uint64_t hash);
+
+/*
+ * New sequence of num_tokens tokens whose first num_hashes full blocks have
+ * the given chained hashes: the longest run of leading blocks found in the
+ * cache is reused (*num_hits of them, refcount + 1 each), the rest are taken
+ * fresh.  PKV_ERR_OOM (nothing taken) if the pool is short.
+ */
+pkv_status pkv_alloc_new_seq_cached(pkv_alloc *a, const uint64_t *block_hashes, int num_hashes,
+                                    int64_t num_tokens, int32_t *out_blocks, int capacity, int *n,
+                                    int *num_hits);
+
 #ifdef __cplusplus
 }
 #endif

@@ -292,7 +292,6 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     constexpr int kHalfBytes = Shape::kHalfBytes;
     constexpr int kTileBytes = Shape::kTileBytes;
     constexpr int kStageBytes = Shape::kStageBytes;
-    constexpr int MT = BS / 16;   // 16-token row tiles per block
     constexpr int KS = D / 16;    // 16-wide column tiles of the head dimension
     static_assert(BS % 16 == 0 && D % 64 == 0, "tile shape");
 

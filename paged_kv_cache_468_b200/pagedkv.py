@@ -96,6 +96,15 @@ def lib() -> ctypes.CDLL:
         L.pkv_alloc_append.argtypes = [P, pi32, i32, pint, i64, i64, pi32, pi32, pint]
         L.pkv_alloc_free.restype = i32
         L.pkv_alloc_free.argtypes = [P, pi32, i32]
+        L.pkv_block_hash.restype = u64
+        L.pkv_block_hash.argtypes = [u64, pi32, i32]
+        L.pkv_alloc_cache_insert.restype = i32
+        L.pkv_alloc_cache_insert.argtypes = [P, u64, ctypes.c_int32]
+        L.pkv_alloc_cache_lookup.restype = ctypes.c_int32
+        L.pkv_alloc_cache_lookup.argtypes = [P, u64]
+        L.pkv_alloc_new_seq_cached.restype = i32
+        L.pkv_alloc_new_seq_cached.argtypes = [P, ctypes.POINTER(ctypes.c_uint64), i32, i64, pi32,
+                                               i32, pint, pint]
         _lib = L
         return L
 
@@ -396,3 +405,32 @@ class BlockAllocator:
 
     def free(self, blocks: list) -> None:
         _check(lib().pkv_alloc_free(self._h, self._arr(blocks), len(blocks)), "pkv_alloc_free")
+
+    # ---- automatic prefix caching ----
+    def block_hashes(self, tokens: list) -> list:
+        """Chained hashes of the full blocks of a token list."""
+        out, parent, bs = [], 0, self.block_size
+        for i in range(len(tokens) // bs):
+            chunk = self._arr(tokens[i * bs:(i + 1) * bs])
+            parent = int(lib().pkv_block_hash(parent, chunk, bs))
+            out.append(parent)
+        return out
+
+    def cache_insert(self, block_hash: int, block: int) -> None:
+        _check(lib().pkv_alloc_cache_insert(self._h, int(block_hash), int(block)),
+               "pkv_alloc_cache_insert")
+
+    def cache_lookup(self, block_hash: int) -> int:
+        return int(lib().pkv_alloc_cache_lookup(self._h, int(block_hash)))
+
+    def new_seq_cached(self, tokens: list) -> tuple:
+        """(blocks, cached leading blocks reused) for a prompt of `tokens`."""
+        hashes = self.block_hashes(tokens)
+        cap = -(-len(tokens) // self.block_size)
+        arr = self._arr([], cap)
+        harr = (ctypes.c_uint64 * max(1, len(hashes)))(*hashes)
+        n, hits = ctypes.c_int(0), ctypes.c_int(0)
+        _check(lib().pkv_alloc_new_seq_cached(self._h, harr, len(hashes), len(tokens), arr, cap,
+                                              ctypes.byref(n), ctypes.byref(hits)),
+               "pkv_alloc_new_seq_cached")
+        return [arr[i] for i in range(n.value)], hits.value

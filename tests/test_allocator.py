@@ -152,3 +152,88 @@ def test_random_lifecycle_conserves_blocks():
         if step % 100 == 0:
             conservation(a, [b for b, _ in seqs.values()])
     conservation(a, [b for b, _ in seqs.values()])
+
+
+# ---- automatic prefix caching ------------------------------------------------
+
+def _register(a, blocks, tokens):
+    for h, b in zip(a.block_hashes(tokens), blocks):
+        a.cache_insert(h, b)
+
+
+def test_block_hash_chains_the_prefix():
+    a = BlockAllocator(8, 4)
+    h1 = a.block_hashes([1, 2, 3, 4, 5, 6, 7, 8])
+    h2 = a.block_hashes([9, 9, 9, 9, 5, 6, 7, 8])     # same 2nd block, different prefix
+    h3 = a.block_hashes([1, 2, 3, 4, 5, 6, 7, 8, 0])  # trailing partial block not hashed
+    assert len(h1) == 2 and h1 == h3
+    assert h1[1] != h2[1] and h1[0] != h2[0]
+    assert all(h != 0 for h in h1 + h2)
+
+
+def test_same_prompt_reuses_cached_blocks():
+    a = BlockAllocator(64, 16, shuffle_seed=3)
+    prompt = list(range(1000, 1000 + 50))             # 3 full blocks + 2 tokens
+    s1, hits1 = a.new_seq_cached(prompt)
+    assert hits1 == 0 and len(s1) == 4
+    _register(a, s1, prompt)                          # after its K/V are written
+    s2, hits2 = a.new_seq_cached(prompt)
+    assert hits2 == 3 and s2[:3] == s1[:3] and s2[3] != s1[3]
+    for b in s1[:3]:
+        assert a.refcount(b) == 2
+    other = prompt[:20] + [7] * 30                    # shares only the first block
+    s3, hits3 = a.new_seq_cached(other)
+    assert hits3 == 1 and s3[0] == s1[0] and s3[1] not in s1
+    conservation(a, [s1, s2, s3])
+
+
+def test_released_cached_blocks_are_revived_or_evicted_lru():
+    a = BlockAllocator(6, 4, shuffle_seed=5)
+    p = [1] * 8                                       # 2 full blocks
+    q = [2] * 8
+    sp, _ = a.new_seq_cached(p)
+    _register(a, sp, p)
+    sq, _ = a.new_seq_cached(q)
+    _register(a, sq, q)
+    a.free(sp)                                        # released first
+    a.free(sq)
+    assert a.num_free == 6                            # free + evictable
+    for b in sp + sq:
+        assert a.refcount(b) == 0
+    again, hits = a.new_seq_cached(q)                 # revived, not recomputed
+    assert hits == 2 and again == sq
+    fresh = a.new_seq(16)                             # needs 4: 2 free + 2 evicted (p's)
+    assert sorted(set(fresh) & set(sp)) == sorted(sp)
+    assert a.cache_lookup(a.block_hashes(p)[0]) == -1  # p's entries were dropped
+    with pytest.raises(PagedKVError) as e:
+        a.new_seq(4)
+    assert e.value.status == pagedkv.ERR_OOM
+    conservation(a, [again, fresh])
+
+
+def test_cache_random_workload_conserves_blocks():
+    rng = random.Random(11)
+    a = BlockAllocator(200, 8, shuffle_seed=11)
+    prompts = [[rng.randrange(50) for _ in range(rng.randrange(8, 80))] for _ in range(12)]
+    live = []
+    for step in range(600):
+        if live and rng.random() < 0.45:
+            a.free(live.pop(rng.randrange(len(live))))
+        else:
+            base = rng.choice(prompts)
+            toks = base[:rng.randrange(1, len(base) + 1)] + [rng.randrange(50) for _ in range(rng.randrange(0, 9))]
+            try:
+                blocks, hits = a.new_seq_cached(toks)
+            except PagedKVError as e:
+                assert e.status == pagedkv.ERR_OOM
+                continue
+            _register(a, blocks, toks)
+            assert len(blocks) == -(-len(toks) // 8)
+            live.append(blocks)
+        refs = {}
+        for t in live:
+            for b in t:
+                refs[b] = refs.get(b, 0) + 1
+        for b, r in refs.items():
+            assert a.refcount(b) == r
+        assert a.num_free + len(refs) == 200
