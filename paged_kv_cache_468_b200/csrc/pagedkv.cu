@@ -705,7 +705,7 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int kPrefillWarps = 8;   // consumer warps: 64 query rows per CTA
+constexpr int kPrefillWarps = 4;   // consumer warps: 32 query rows per CTA, 3 CTAs per SM
 
 template <int D, int BS, bool BF16>
 cudaError_t launch_prefill(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::PrefillArgs &p,

@@ -571,7 +571,10 @@ struct CascadeArgs {
 };
 
 template <int D, int BS, bool BF16, int NWQ, int S>
-__global__ void __launch_bounds__((NWQ + 1) * 32, 1)
+// Up to 4 consumer warps the kernel is held to 128 registers so that three
+// CTAs share an SM: the consumers are latency-bound (mma, shuffles, waits)
+// and need the extra warps; 8-warp CTAs would spill at that limit.
+__global__ void __launch_bounds__((NWQ + 1) * 32, (NWQ <= 4 ? 3 : 1))
 prefix_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      const CascadeArgs a)
 {
@@ -848,7 +851,9 @@ struct PrefillArgs {
 };
 
 template <int D, int BS, bool BF16, int NWQ, int S>
-__global__ void __launch_bounds__((NWQ + 1) * 32, 1)
+// Held to 128 registers (3 CTAs of 4 consumer warps per SM) for the same
+// reason as the prefix pass above.
+__global__ void __launch_bounds__((NWQ + 1) * 32, 3)
 prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                const PrefillArgs a)
 {
