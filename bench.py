@@ -560,7 +560,7 @@ def run_other_op(args, cfg, world, rank, local):
                               "peak": peak, "unit": "TFLOP/s",
                               "frac": round(flops / (ms * 1e-3) / 1e12 / peak, 4),
                               "peak_source": "MEASURED_PEAKS.json bf16_tflops (cuBLAS bf16)",
-                              "note": "mma.sync m16n8k16 (legacy tensor path)"})
+                              "note": "tcgen05.mma (TMEM accumulators), 128 query rows x 64-key tiles"})
         line["config"].update(chunk=args.chunk, query_tokens=T)
     else:
         n = min(args.pairs, NB // 2)

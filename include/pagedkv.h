@@ -211,9 +211,13 @@ pkv_status pkv_paged_attention_decode(const void *query, const void *key_cache,
  *
  * Query token i of sequence b sits at position L_b - C_b + i and attends
  * causally over the sequence's tokens 0 .. L_b - C_b + i.  One CTA per tile of
- * 64 (token, query head) rows of one sequence and kv head; a producer warp
- * streams the blocks the tile needs into shared memory (TMA), eight consumer
- * warps apply their rows to each block with mma.sync.  A chunk longer than
+ * 128 (token, query head) rows of one sequence and kv head; its blocks are
+ * streamed into shared memory (TMA) 64 keys at a time and both products
+ * (Q K^T and P V) run on the tcgen05 tensor cores with f32 accumulators in
+ * tensor memory.  The attention weights P are rounded to the cache dtype
+ * before P V; the row sums are taken over those rounded weights.  The
+ * group size (num_heads / num_kv_heads) is at most 8, as for decode.  A
+ * chunk longer than
  * its context or than max_query_len, or outside the query rows, sets
  * PKV_DEVFLAG_CONTEXT_RANGE (such a chunk is clamped or skipped).
  */

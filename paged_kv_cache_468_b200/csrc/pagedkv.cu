@@ -16,6 +16,7 @@
 
 #include "pagedkv.h"
 #include "pkv_kernels.cuh"
+#include "pkv_prefill.cuh"
 
 namespace {
 
@@ -86,6 +87,28 @@ pkv_status make_cache_map(CUtensorMap *map, const void *base, int64_t num_blocks
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+    return PKV_OK;
+}
+
+// The query [T, Hq, D] seen as {D, Hq, T}; a box is 64 columns x the G heads
+// of one kv head x `tokens` query tokens: rows (token, head) of 128 bytes,
+// 128-byte swizzle, the prefill CTA's Q tile.  Rows past T read as zero.
+pkv_status make_query_map(CUtensorMap *map, const void *base, int64_t T, int Hq, int D, int G,
+                          int tokens, pkv_dtype dt)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)tokens};
+    cuuint32_t estride[3] = {1, 1, 1};
+    CUresult r = enc(map, dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                     3, const_cast<void *>(base), dims, strides, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (query) failed (CUresult %d)", (int)r);
     return PKV_OK;
 }
 
@@ -705,34 +728,33 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int kPrefillWarps = 4;   // consumer warps: 32 query rows per CTA, 3 CTAs per SM
-
 template <int D, int BS, bool BF16>
-cudaError_t launch_prefill(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::PrefillArgs &p,
-                           int max_query_len, cudaStream_t st)
+cudaError_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                           const pkv::PrefillArgs &p, int max_query_len, cudaStream_t st)
 {
-    constexpr int NWQ = kPrefillWarps;
-    constexpr int S = BS == 16 ? 4 : 3;
-    using Shape = pkv::DecodeShape<D, BS, 1, S>;
-    constexpr int smem = S * Shape::kStageBytes + 1024;
-    auto kern = pkv::prefill_kernel<D, BS, BF16, NWQ, S>;
+    constexpr int smem = pkv::PfShape<D>::kSmemBytes;
+    auto kern = pkv::prefill_tc_kernel<D, BS, BF16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)   // two CTAs (and their TMEM) per SM
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess)
         return e;
-    const int64_t rows = (int64_t)max_query_len * p.group;
-    const dim3 grid((unsigned)((rows + NWQ * 8 - 1) / (NWQ * 8)), (unsigned)p.num_kv_heads,
-                    (unsigned)p.batch);
-    return launch_pdl(kern, grid, dim3((NWQ + 1) * 32), smem, st, mk, mv, p);
+    const int tokens_per_cta = pkv::kPfRows / p.group;
+    const dim3 grid((unsigned)((max_query_len + tokens_per_cta - 1) / tokens_per_cta),
+                    (unsigned)p.num_kv_heads, (unsigned)p.batch);
+    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, mk, mv, p);
 }
 
 template <bool BF16>
-cudaError_t dispatch_prefill(int D, int bs, const CUtensorMap &mk, const CUtensorMap &mv,
-                             const pkv::PrefillArgs &p, int max_query_len, cudaStream_t st)
+cudaError_t dispatch_prefill(int D, int bs, const CUtensorMap &mq, const CUtensorMap &mk,
+                             const CUtensorMap &mv, const pkv::PrefillArgs &p, int max_query_len,
+                             cudaStream_t st)
 {
-    if (D == 64 && bs == 16) return launch_prefill<64, 16, BF16>(mk, mv, p, max_query_len, st);
-    if (D == 64 && bs == 32) return launch_prefill<64, 32, BF16>(mk, mv, p, max_query_len, st);
-    if (D == 128 && bs == 16) return launch_prefill<128, 16, BF16>(mk, mv, p, max_query_len, st);
-    return launch_prefill<128, 32, BF16>(mk, mv, p, max_query_len, st);
+    if (D == 64 && bs == 16) return launch_prefill<64, 16, BF16>(mq, mk, mv, p, max_query_len, st);
+    if (D == 64 && bs == 32) return launch_prefill<64, 32, BF16>(mq, mk, mv, p, max_query_len, st);
+    if (D == 128 && bs == 16) return launch_prefill<128, 16, BF16>(mq, mk, mv, p, max_query_len, st);
+    return launch_prefill<128, 32, BF16>(mq, mk, mv, p, max_query_len, st);
 }
 
 }  // namespace
@@ -766,7 +788,11 @@ extern "C" pkv_status pkv_paged_attention_prefill(
         return fail(PKV_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
         return fail(PKV_ERR_MISALIGNED, "query/cache/out pointers must be 16-byte aligned");
-    CUtensorMap mk, mv;
+    CUtensorMap mq, mk, mv;
+    const int group = num_heads / num_kv_heads;
+    if ((s = make_query_map(&mq, query, num_tokens, num_heads, head_dim, group, pkv::kPfRows / group,
+                            dtype)) != PKV_OK)
+        return s;
     if ((s = make_cache_map(&mk, key_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
         return s;
     if ((s = make_cache_map(&mv, value_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
@@ -788,10 +814,10 @@ extern "C" pkv_status pkv_paged_attention_prefill(
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = dtype == PKV_BF16
-                        ? dispatch_prefill<true>(head_dim, block_size, mk, mv, p, max_query_len, st)
-                        : dispatch_prefill<false>(head_dim, block_size, mk, mv, p, max_query_len, st);
+                        ? dispatch_prefill<true>(head_dim, block_size, mq, mk, mv, p, max_query_len, st)
+                        : dispatch_prefill<false>(head_dim, block_size, mq, mk, mv, p, max_query_len, st);
     if (e != cudaSuccess)
-        return cuda_fail(e, "prefill_kernel launch");
+        return cuda_fail(e, "prefill_tc_kernel launch");
     return PKV_OK;
 }
 

@@ -134,14 +134,12 @@ __global__ void kv_write_kernel(const uint4 *__restrict__ key, const uint4 *__re
 //   S^T[t, n] = sum_d K[t, d] Q[n, d]            (mma.sync m16n8k16, fp32)
 //   online softmax per column n
 //   O^T[d, n] += sum_t V[t, d] P[t, n]
-// CAUSAL: token t of the block is also masked for column j when t > lim[j]
-// (the lane's columns 2c, 2c+1; lim relative to the block's first token).
-template <int D, int BS, bool BF16, bool CAUSAL = false>
+template <int D, int BS, bool BF16>
 __device__ __forceinline__ void attend_block(uint32_t sk, uint32_t sv, int valid,
                                              const uint32_t (&qf)[D / 16][2], float scale_log2,
                                              float (&m_run)[2], float (&l_run)[2],
                                              float (&acc_hi)[D / 16][4], float (&acc_lo)[D / 16][4],
-                                             int lane, const int (&lim)[2] = {0, 0})
+                                             int lane)
 {
     constexpr int MT = BS / 16;
     constexpr int KS = D / 16;
@@ -177,8 +175,7 @@ __device__ __forceinline__ void attend_block(uint32_t sk, uint32_t sv, int valid
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = mt * 16 + (lane >> 2) + (i >= 2 ? 8 : 0);
-            const bool ok = t < valid && (!CAUSAL || t <= lim[i & 1]);
-            const float v = ok ? sc[mt][i] * scale_log2 : kNegInf;
+            const float v = t < valid ? sc[mt][i] * scale_log2 : kNegInf;
             sc[mt][i] = v;
             mx[i & 1] = fmaxf(mx[i & 1], v);
         }
@@ -818,248 +815,6 @@ lse_merge_cascade_kernel(const CascadeArgs c, const float *__restrict__ sm, cons
         fold(__ldg(sm + rec), __ldg(sl + rec), __ldg(so + rec * D + d));
     }
     out[row * D + d] = to_storage<BF16>(den > 0.f ? num / den : 0.f);
-}
-
-// ---------------------------------------------------------------------------
-// Chunked prefill over the paged cache
-// ---------------------------------------------------------------------------
-// Sequence b brings C_b = query_start[b+1] - query_start[b] new tokens, the
-// last C_b of its L_b = context_lens[b] cached tokens (their K/V written
-// through slot_mapping beforehand); query token i sits at position
-// L_b - C_b + i and attends causally over tokens 0 .. L_b - C_b + i.  One CTA
-// per (row tile, kv head, sequence), rows = (token, head of the GQA group)
-// pairs, NWQ consumer warps of 8 rows each; a producer warp streams the
-// blocks the tile needs (through its last row's position) into a CTA-wide
-// TMA ring.  Rows past a block's end or past a column's position are masked;
-// V rows past the context end in the last block are zeroed once (warp 0,
-// then a consumer-only named barrier) so masked weights stay exactly zero.
-struct PrefillArgs {
-    const uint16_t *query;           // [T, Hq, D], T = query_start[batch]
-    const int32_t *query_start;      // [batch + 1]
-    const int32_t *block_tables;     // [batch, max_blocks]
-    const int32_t *context_lens;     // [batch]
-    uint16_t *out;                   // [T, Hq, D]
-    int batch;
-    int num_tokens;                  // T: rows of query / out
-    int max_query_len;               // chunks longer than this are not covered by the grid
-    int max_blocks;
-    int num_heads;
-    int num_kv_heads;
-    int group;
-    int num_blocks;
-    float scale_log2;
-};
-
-template <int D, int BS, bool BF16, int NWQ, int S>
-// Held to 128 registers (3 CTAs of 4 consumer warps per SM) for the same
-// reason as the prefix pass above.
-__global__ void __launch_bounds__((NWQ + 1) * 32, 3)
-prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-               const PrefillArgs a)
-{
-    using Shape = DecodeShape<D, BS, 1, S>;
-    constexpr int kHalfBytes = Shape::kHalfBytes;
-    constexpr int kTileBytes = Shape::kTileBytes;
-    constexpr int kStageBytes = Shape::kStageBytes;
-    constexpr int KS = D / 16;
-    constexpr int R = NWQ * 8;                  // query rows per CTA
-
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[S];
-    __shared__ __align__(8) uint64_t empty[S];
-    __shared__ __align__(8) uint64_t last_ready;   // last block's V tail zeroed
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t ring_s = smem_addr(smem);
-
-    const int tile = blockIdx.x;
-    const int kvh = blockIdx.y;
-    const int b = blockIdx.z;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int G = a.group;
-
-    if (threadIdx.x == 0) {
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-            mbar_init(smem_addr(&full[s]), 1);
-            mbar_init(smem_addr(&empty[s]), NWQ);
-        }
-        mbar_init(smem_addr(&last_ready), 1);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-    }
-    fence_mbar_init();
-    __syncthreads();
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;");
-
-    const int q0 = __ldg(a.query_start + b);
-    int C = __ldg(a.query_start + b + 1) - q0;
-    int L = __ldg(a.context_lens + b);
-    const int span = a.max_blocks * BS;
-    if (q0 < 0 || C < 0 || q0 + C > a.num_tokens || C > a.max_query_len || L < 0 || L > span ||
-        C > L) {
-        if (threadIdx.x == 0 && tile == 0 && kvh == 0)
-            raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
-        L = L < 0 ? 0 : (L > span ? span : L);
-        if (q0 < 0 || C < 0 || q0 + C > a.num_tokens)
-            C = 0;                                  // rows outside query/out: skip the sequence
-        C = min(C, min(L, a.max_query_len));
-    }
-    const int rows = C * G;
-    const int row0 = tile * R;
-    if (row0 >= rows)
-        return;
-    const int last_tok = min(C, (row0 + R + G - 1) / G) - 1;   // last query token of the tile
-    const int p_max = L - C + last_tok;                          // its position
-    const int nblk = p_max / BS + 1;
-
-    if (warp == NWQ) {
-        // ---- producer ----
-        const int32_t *trow = a.block_tables + (size_t)b * a.max_blocks;
-        const uint64_t policy = policy_evict_normal();   // tiles of one sequence reread the blocks
-        int ids = 0;
-        for (int k = 0; k < nblk; ++k) {
-            const int s = k % S;
-            if (k >= S) {
-                const bool ok = mbar_wait_bounded(smem_addr(&empty[s]), (uint32_t)(((k / S) - 1) & 1),
-                                                  kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0)
-                        raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-                    break;
-                }
-            }
-            if ((k & 31) == 0)
-                ids = k + lane < nblk ? __ldg(trow + k + lane) : 0;
-            int blk = __shfl_sync(0xffffffffu, ids, k & 31);
-            if ((unsigned)blk >= (unsigned)a.num_blocks) {
-                if (lane == 0)
-                    raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
-                blk = 0;
-            }
-            if (lane == 0) {
-                const uint32_t bar = smem_addr(&full[s]);
-                const uint32_t dk = ring_s + (uint32_t)(s * kStageBytes);
-                mbar_arrive_expect_tx(bar, kStageBytes);
-#pragma unroll
-                for (int h = 0; h < Shape::kHalves; ++h) {
-                    tma_load_3d(dk + h * kHalfBytes, &tm_k, bar, h * 64, kvh, blk * BS, policy);
-                    tma_load_3d(dk + kTileBytes + h * kHalfBytes, &tm_v, bar, h * 64, kvh, blk * BS,
-                                policy);
-                }
-            }
-        }
-        // the context's last block, when partial: zero its V rows past the end
-        // once the tile has landed, then release the consumers for that block
-        const int k_last = nblk - 1;
-        const int valid_last = min(BS, L - k_last * BS);
-        if (valid_last < BS) {
-            const int s = k_last % S;
-            const bool ok = mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((k_last / S) & 1),
-                                              kWaitLimitNs);
-            if (__all_sync(0xffffffffu, ok)) {
-                uint8_t *vt = smem + (size_t)s * kStageBytes + kTileBytes;
-                const int per_half = (BS - valid_last) * 8;
-                for (int i = lane; i < Shape::kHalves * per_half; i += 32) {
-                    const int h = i / per_half;
-                    const int r = i - h * per_half;
-                    *reinterpret_cast<uint4 *>(vt + h * kHalfBytes + (valid_last + (r >> 3)) * 128 +
-                                               (r & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
-                }
-            } else if (lane == 0) {
-                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(smem_addr(&last_ready));
-        }
-        return;
-    }
-
-    // ---- consumers: warp w owns rows row0 + 8w + n: token i = row / G, head g = row % G ----
-    const int c = lane & 3;
-    int pos[2];                                  // positions of the lane's columns 2c, 2c+1
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int row = row0 + warp * 8 + 2 * c + j;
-        pos[j] = row < rows ? L - C + row / G : p_max;   // rows past the chunk: never masked
-    }
-    uint32_t qf[KS][2];
-    {
-        const int row = row0 + warp * 8 + (lane >> 2);
-        const bool ok = row < rows;
-        const int i = ok ? row / G : 0;
-        const int g = ok ? row - (row / G) * G : 0;
-        const uint32_t *q32 = reinterpret_cast<const uint32_t *>(
-            a.query + ((size_t)(q0 + i) * a.num_heads + (size_t)kvh * G + g) * D);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qf[ks][0] = ok ? __ldg(q32 + ks * 8 + c) : 0u;
-            qf[ks][1] = ok ? __ldg(q32 + ks * 8 + 4 + c) : 0u;
-        }
-    }
-    float m_run[2] = {kNegInf, kNegInf};
-    float l_run[2] = {0.f, 0.f};
-    float acc_hi[KS][4], acc_lo[KS][4];
-#pragma unroll
-    for (int dt = 0; dt < KS; ++dt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc_hi[dt][i] = 0.f;
-            acc_lo[dt][i] = 0.f;
-        }
-    int consumed = 0;
-    for (int k = 0; k < nblk; ++k) {
-        const int s = k % S;
-        const int valid = min(BS, L - k * BS);
-        // a partial block (only the context's last) is released by the producer
-        // after it zeroed the V rows past the end
-        const bool got = valid < BS
-                             ? mbar_wait_bounded(smem_addr(&last_ready), 0u, kWaitLimitNs)
-                             : mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((k / S) & 1),
-                                                 kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, got)) {
-            if (lane == 0)
-                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-            break;
-        }
-        const uint32_t sk = ring_s + (uint32_t)(s * kStageBytes);
-        consumed = k + 1;
-        const int lim[2] = {pos[0] - k * BS, pos[1] - k * BS};
-        attend_block<D, BS, BF16, true>(sk, sk + kTileBytes, valid, qf, a.scale_log2, m_run, l_run,
-                                        acc_hi, acc_lo, lane, lim);
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(smem_addr(&empty[s]));
-    }
-    for (int k = consumed; k < nblk && k < consumed + S; ++k)
-        mbar_wait_bounded(smem_addr(&full[k % S]), (uint32_t)((k / S) & 1), kWaitLimitNs / 8);
-
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 4);
-        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 8);
-        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 16);
-    }
-    const int r = lane >> 2;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int row = row0 + warp * 8 + 2 * c + j;
-        if (row >= rows)
-            continue;
-        const int i = row / G;
-        const int g = row - i * G;
-        const size_t orow = (size_t)(q0 + i) * a.num_heads + (size_t)kvh * G + g;
-        const float inv = l_run[j] > 0.f ? 1.f / l_run[j] : 0.f;
-#pragma unroll
-        for (int dt = 0; dt < KS; ++dt) {
-            a.out[orow * D + dt * 16 + r] = to_storage<BF16>((acc_hi[dt][j] + acc_lo[dt][j]) * inv);
-            a.out[orow * D + dt * 16 + r + 8] =
-                to_storage<BF16>((acc_hi[dt][2 + j] + acc_lo[dt][2 + j]) * inv);
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------

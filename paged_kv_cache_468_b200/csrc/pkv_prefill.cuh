@@ -1,0 +1,437 @@
+// pkv_prefill.cuh -- chunked prefill over the paged KV cache on the
+// 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory).
+//
+// Sequence b brings C_b = query_start[b+1] - query_start[b] new tokens, the
+// last C_b of its L_b = context_lens[b] cached tokens (their K/V were written
+// through slot_mapping beforehand, "大模型推理框架 vLLM 源码解析 一",
+// section 三); query token i sits at position L_b - C_b + i and attends
+// causally over tokens 0 .. L_b - C_b + i of its paged cache.
+//
+// One CTA per (row tile, kv head, sequence).  A row is a (query token, head
+// of the kv head's GQA group) pair, 128 rows per CTA (the M of every MMA).
+// Keys are taken 64 at a time (a "key tile": 64 / block_size cache blocks
+// located through the block table, exactly as the decode kernels do):
+//
+//   S_j  = Q K_j^T        tcgen05.mma, Q and K_j in shared memory, S in TMEM
+//   P_j  = 2^(S_j*scale*log2e - m)    one row per softmax thread, bf16/f16
+//                                      into shared memory
+//   O   += P_j V_j         tcgen05.mma, O in TMEM (V read MN-major)
+//
+// The running row maximum m is only moved when a tile's maximum exceeds it
+// by more than 2^8 (P then stays <= 256); O and the row sum are rescaled by
+// the softmax warps at that point, so the result equals the one-pass softmax
+// up to rounding.  Warp roles: 0-3 softmax + epilogue (warp w owns TMEM lanes
+// 32w..32w+31), 4 loads Q and the K ring, 5 allocates TMEM and issues every
+// MMA, 6 loads the V ring and clears V rows past the last visible key (so
+// masked weights meet finite values).  Every wait is bounded; on a time-out
+// the CTA records PKV_DEVFLAG_WAIT_TIMEOUT, lets in-flight copies and MMAs
+// finish and frees its TMEM.
+#pragma once
+
+#include "pkv_kernels.cuh"
+
+namespace pkv {
+
+struct PrefillArgs {
+    const uint16_t *query;           // [T, Hq, D], T = query_start[batch]
+    const int32_t *query_start;      // [batch + 1]
+    const int32_t *block_tables;     // [batch, max_blocks]
+    const int32_t *context_lens;     // [batch]
+    uint16_t *out;                   // [T, Hq, D]
+    int batch;
+    int num_tokens;                  // T: rows of query / out
+    int max_query_len;               // chunks longer than this are not covered by the grid
+    int max_blocks;
+    int num_heads;
+    int num_kv_heads;
+    int group;
+    int num_blocks;
+    float scale_log2;
+};
+
+constexpr int kPfRows = 128;             // query rows per CTA (MMA M)
+constexpr int kPfKeys = 64;              // keys per tile (N of Q K^T, K of P V)
+constexpr int kPfThreads = 224;          // 7 warps
+constexpr uint32_t kPfTmemCols = 256;    // S: 2 x 64 columns, O: D columns at 128
+
+template <int D>
+struct PfShape {
+    static constexpr int kHalves = D / 64;                  // 128-byte column halves
+    static constexpr int kQHalf = kPfRows * 128;            // one half of Q: 128 rows x 128 B
+    static constexpr int kKVHalf = kPfKeys * 128;           // one half of a K or V tile
+    static constexpr int kQBytes = kHalves * kQHalf;
+    static constexpr int kKVBytes = kHalves * kKVHalf;
+    static constexpr int kPBytes = kPfRows * kPfKeys * 2;   // 128 rows x 128 B
+    static constexpr int kQOff = 0;
+    static constexpr int kKOff = kQOff + kQBytes;           // 2 stages
+    static constexpr int kVOff = kKOff + 2 * kKVBytes;      // 2 stages
+    static constexpr int kPOff = kVOff + 2 * kKVBytes;
+    static constexpr int kDataBytes = kPOff + kPBytes;
+    // + 1024 so that the data can start on a 1024-byte boundary; the barriers
+    // sit in whichever end of that slack has room
+    static constexpr int kSmemBytes = kDataBytes + 1024;
+};
+
+// mbarrier slots
+enum PfBar {
+    kBarQFull = 0,
+    kBarKFull = 1,     // 2
+    kBarKEmpty = 3,    // 2
+    kBarVFull = 5,     // 2
+    kBarVEmpty = 7,    // 2
+    kBarSFull = 9,     // 2
+    kBarPFull = 11,
+    kBarODone = 12,
+    kBarVTail = 13,
+    kBarDrain = 14,
+    kBarTmemSlot = 15,   // not a barrier: the TMEM base address
+    kNumPfBars = 16
+};
+
+template <int D, int BS, bool BF16>
+__global__ void __launch_bounds__(kPfThreads, 2)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a)
+{
+    using Sh = PfShape<D>;
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
+    static_assert(kPfKeys % BS == 0, "whole blocks per key tile");
+    static_assert(kPfKeys + D <= (int)kPfTmemCols, "TMEM columns");
+    constexpr int KS = D / 16;               // k-steps of Q K^T
+    constexpr int KV_STEPS = kPfKeys / 16;   // k-steps of P V
+    constexpr int BPT = kPfKeys / BS;        // cache blocks per key tile
+
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw_s = smem_addr(smem_raw);
+    const uint32_t data_s = (raw_s + 1023u) & ~1023u;
+    uint8_t *data = smem_raw + (data_s - raw_s);
+    const uint32_t bars_s = data_s - raw_s >= kNumPfBars * 8 ? raw_s : data_s + Sh::kDataBytes;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + (bars_s - raw_s));
+    auto bar = [&](int i) { return bars_s + 8u * (uint32_t)i; };
+
+    const int tile = blockIdx.x;
+    const int kvh = blockIdx.y;
+    const int b = blockIdx.z;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int G = a.group;
+    const int TT = kPfRows / G;   // query tokens per CTA
+    const int R = TT * G;         // rows in use (128 when G divides 128)
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar(kBarQFull), 1);
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(kBarKFull + s), 1);
+            mbar_init(bar(kBarKEmpty + s), 1);
+            mbar_init(bar(kBarVFull + s), 1);
+            mbar_init(bar(kBarVEmpty + s), 1);
+            mbar_init(bar(kBarSFull + s), 1);
+        }
+        mbar_init(bar(kBarPFull), 128);
+        mbar_init(bar(kBarODone), 1);
+        mbar_init(bar(kBarVTail), 1);
+        mbar_init(bar(kBarDrain), 1);
+        prefetch_tensormap(&tm_q);
+        prefetch_tensormap(&tm_k);
+        prefetch_tensormap(&tm_v);
+    }
+    fence_mbar_init();
+    __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
+
+    const int q0 = __ldg(a.query_start + b);
+    int C = __ldg(a.query_start + b + 1) - q0;
+    int L = __ldg(a.context_lens + b);
+    const int span = a.max_blocks * BS;
+    if (q0 < 0 || C < 0 || q0 + C > a.num_tokens || C > a.max_query_len || L < 0 || L > span ||
+        C > L) {
+        if (threadIdx.x == 0 && tile == 0 && kvh == 0)
+            raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+        L = L < 0 ? 0 : (L > span ? span : L);
+        if (q0 < 0 || C < 0 || q0 + C > a.num_tokens)
+            C = 0;                                  // rows outside query/out: skip the sequence
+        C = min(C, min(L, a.max_query_len));
+    }
+    const int rows = C * G;
+    const int row0 = tile * R;
+    if (row0 >= rows)
+        return;                                     // whole CTA, before TMEM is touched
+    const int i0 = tile * TT;                       // first query token of the CTA
+    const int last_tok = min(C, i0 + TT) - 1;
+    const int p_max = L - C + last_tok;             // last key any row of the CTA sees
+    const int pos0 = L - C + i0;                    // ... and the first row's last key
+    const int nt = p_max / kPfKeys + 1;             // key tiles
+    const int nblk = p_max / BS + 1;                // cache blocks read
+
+    // ---- tensor memory ----
+    if (warp == 5) {
+        tmem_alloc(bar(kBarTmemSlot), kPfTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(&bars[kBarTmemSlot]);
+    const uint32_t tO = tmem + 2 * kPfKeys;         // O columns
+
+    const uint32_t sQ = data_s + Sh::kQOff;
+    const uint32_t sK = data_s + Sh::kKOff;
+    const uint32_t sV = data_s + Sh::kVOff;
+    const uint32_t sP = data_s + Sh::kPOff;
+
+    if (warp == 4 || warp == 6) {
+        // ---- loads: warp 4 Q and the K ring, warp 6 the V ring ----
+        const bool is_k = warp == 4;
+        const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+        const int full0 = is_k ? kBarKFull : kBarVFull;
+        const int empty0 = is_k ? kBarKEmpty : kBarVEmpty;
+        const uint32_t ring = is_k ? sK : sV;
+        int issued = 0;
+        if (lane == 0) {
+            const uint64_t policy = policy_evict_normal();   // the sequence's other CTAs reread them
+            const int32_t *trow = a.block_tables + (size_t)b * a.max_blocks;
+            if (is_k) {
+                mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(Sh::kHalves * R * 128));
+#pragma unroll
+                for (int h = 0; h < Sh::kHalves; ++h)
+                    tma_load_3d(sQ + h * Sh::kQHalf, &tm_q, bar(kBarQFull), h * 64, kvh * G, q0 + i0,
+                                policy);
+            }
+            for (int j = 0; j < nt; ++j) {
+                const int s = j & 1;
+                if (j >= 2 &&
+                    !mbar_wait_bounded(bar(empty0 + s), (uint32_t)(((j >> 1) - 1) & 1), kWaitLimitNs)) {
+                    raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+                    break;
+                }
+                const int kb0 = j * BPT;
+                const int nb = min(BPT, nblk - kb0);
+                mbar_arrive_expect_tx(bar(full0 + s), (uint32_t)(nb * BS * D * 2));
+                for (int i = 0; i < nb; ++i) {
+                    int blk = __ldg(trow + kb0 + i);
+                    if ((unsigned)blk >= (unsigned)a.num_blocks) {
+                        raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
+                        blk = 0;
+                    }
+#pragma unroll
+                    for (int h = 0; h < Sh::kHalves; ++h)
+                        tma_load_3d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
+                                    bar(full0 + s), h * 64, kvh, blk * BS, policy);
+                }
+                issued = j + 1;
+            }
+        }
+        issued = __shfl_sync(0xffffffffu, issued, 0);
+        if (!is_k && issued == nt) {
+            // V rows of the last tile past p_max (the context's tail in its last
+            // block, and blocks never loaded) are cleared once the tile landed
+            const int j = nt - 1;
+            const int s = j & 1;
+            const bool landed = mbar_wait_bounded(bar(kBarVFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
+            if (__all_sync(0xffffffffu, landed)) {
+                const int z0 = p_max + 1 - j * kPfKeys;   // first row to clear, 1 .. 64
+                if (z0 < kPfKeys) {
+                    uint8_t *vt = data + Sh::kVOff + s * Sh::kKVBytes;
+                    const int per_half = (kPfKeys - z0) * 8;   // 16-byte vectors
+                    for (int i = lane; i < Sh::kHalves * per_half; i += 32) {
+                        const int h = i / per_half;
+                        const int r = i - h * per_half;
+                        *reinterpret_cast<uint4 *>(vt + h * Sh::kKVHalf + (z0 + (r >> 3)) * 128 +
+                                                   (r & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                }
+                fence_proxy_async_smem();
+            } else if (lane == 0) {
+                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+            }
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(kBarVTail));
+        }
+        // copies still in flight land before the CTA can exit
+        if (lane == 0) {
+            if (is_k)
+                mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs / 8);
+            for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j)
+                mbar_wait_bounded(bar(full0 + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs / 8);
+        }
+    } else if (warp == 5) {
+        // ---- MMA issue: one thread ----
+        if (lane == 0) {
+            constexpr uint32_t idS = f16_idesc<BF16>(kPfRows, kPfKeys, false);
+            constexpr uint32_t idO = f16_idesc<BF16>(kPfRows, D, true);
+            // S_j = Q K_j^T into S buffer j & 1; Q and K K-major, 128-byte rows
+            auto issue_s = [&](int j) -> bool {
+                const int s = j & 1;
+                if (!mbar_wait_bounded(bar(kBarKFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs))
+                    return false;
+                tc_fence_after();
+                const uint32_t kt = sK + s * Sh::kKVBytes;
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    const uint32_t koff = (uint32_t)((ks & 3) * 32);   // 16 elements = 32 bytes
+                    tc_mma_f16(tmem + s * kPfKeys,
+                               sw128_desc(sQ + (ks >> 2) * Sh::kQHalf + koff, 16, 1024),
+                               sw128_desc(kt + (ks >> 2) * Sh::kKVHalf + koff, 16, 1024), idS,
+                               ks > 0 ? 1u : 0u);
+                }
+                tc_commit(bar(kBarSFull + s));
+                tc_commit(bar(kBarKEmpty + s));
+                return true;
+            };
+            bool ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
+            for (int j = 0; ok && j < nt; ++j) {
+                if (j + 1 < nt && !(ok = issue_s(j + 1)))
+                    break;
+                const int s = j & 1;
+                ok = mbar_wait_bounded(bar(kBarPFull), (uint32_t)(j & 1), kWaitLimitNs) &&
+                     mbar_wait_bounded(bar(kBarVFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
+                     (j + 1 < nt || mbar_wait_bounded(bar(kBarVTail), 0u, kWaitLimitNs));
+                if (!ok)
+                    break;
+                tc_fence_after();
+                // O += P_j V_j: P K-major (keys along its 128-byte rows), V
+                // MN-major (head dim along the rows: halves LBO apart, 8-key
+                // groups 1024 bytes apart)
+                const uint32_t vt = sV + s * Sh::kKVBytes;
+#pragma unroll
+                for (int kk = 0; kk < KV_STEPS; ++kk)
+                    tc_mma_f16(tO, sw128_desc(sP + kk * 32, 16, 1024),
+                               sw128_desc(vt + kk * 16 * 128, Sh::kKVHalf, 1024), idO,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                tc_commit(bar(kBarODone));
+                tc_commit(bar(kBarVEmpty + s));
+            }
+            if (!ok)
+                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+            // every MMA issued has finished before the TMEM is released
+            tc_commit(bar(kBarDrain));
+            mbar_wait_bounded(bar(kBarDrain), 0u, kWaitLimitNs);
+        }
+    } else {
+        // ---- softmax and epilogue: thread = row r of the tile = TMEM lane r ----
+        const int r = warp * 32 + lane;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int grow = row0 + r;                  // row within the sequence
+        const bool real = r < R && grow < rows;
+        const int pos = real ? L - C + grow / G : p_max;
+        float m_used = kNegInf;
+        float l = 0.f;
+        bool ok = true;
+        uint8_t *prow = data + Sh::kPOff + r * 128;
+        for (int j = 0; j < nt; ++j) {
+            const int s = j & 1;
+            ok = mbar_wait_bounded(bar(kBarSFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            uint32_t raw[64];
+            tmem_ld64(tmem + lane_base + s * kPfKeys, raw);
+            float x[64];
+            float mt = kNegInf;
+            const int t0 = j * kPfKeys;
+            if (t0 + kPfKeys - 1 <= pos0) {         // every key visible to every row
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    x[c] = __uint_as_float(raw[c]) * a.scale_log2;
+                    mt = fmaxf(mt, x[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    x[c] = t0 + c <= pos ? __uint_as_float(raw[c]) * a.scale_log2 : kNegInf;
+                    mt = fmaxf(mt, x[c]);
+                }
+            }
+            const bool resc = mt > m_used + 8.f;    // first tile: m_used = -inf
+            const float m_new = resc ? mt : m_used;
+            const float alpha = resc ? ex2(m_used - m_new) : 1.f;
+            const float msub = m_new == kNegInf ? 0.f : m_new;
+            // the row sum is taken over the rounded weights the MMA multiplies,
+            // so the normalised weights sum to one exactly
+            uint32_t pk[32];
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+                pk[c] = pack2<BF16>(ex2(x[2 * c] - msub), ex2(x[2 * c + 1] - msub));
+                const float2 pr = unpack2<BF16>(pk[c]);
+                rs += pr.x + pr.y;
+            }
+            l = l * alpha + rs;
+            m_used = m_new;
+            if (j > 0) {
+                // the P buffer and O belong to P_{j-1} V_{j-1} until it completes
+                ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t o[32];
+                        tmem_ld32(tO + lane_base + c0, o);
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tmem_st32(tO + lane_base + c0, o);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            // P row r into the 128-byte swizzled layout: 16-byte chunk c of the
+            // row goes to chunk c ^ (r & 7)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) =
+                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(kBarPFull));
+        }
+        if (ok)
+            ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((nt - 1) & 1), kWaitLimitNs);
+        if (__all_sync(0xffffffffu, ok)) {
+            tc_fence_after();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int i = real ? grow / G : 0;
+            const int g = real ? grow - i * G : 0;
+            uint4 *orow = reinterpret_cast<uint4 *>(
+                a.out + ((size_t)(q0 + i) * a.num_heads + (size_t)kvh * G + g) * D);
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + lane_base + c0, o);
+                if (real) {
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            w[e] = pack2<BF16>(__uint_as_float(o[8 * v + 2 * e]) * inv,
+                                               __uint_as_float(o[8 * v + 2 * e + 1]) * inv);
+                        orow[c0 / 8 + v] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                }
+            }
+        } else if (lane == 0) {
+            raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+        }
+    }
+
+    // ---- release the tensor memory once every warp is done with it ----
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 5) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, kPfTmemCols);
+    }
+}
+
+}  // namespace pkv

@@ -52,7 +52,7 @@ def test_prefill_ragged_chunks(D, bs, dtype):
     _check(step, q, qs, chunks)
 
 
-@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("G", [1, 3, 4, 6, 8])
 def test_prefill_group_sizes(G):
     lens = [700, 129, 520]
     chunks = [512, 129, 7]
@@ -71,3 +71,24 @@ def test_prefill_last_token_equals_decode():
     dec = pkv.paged_attention_decode(last, d["key_cache"], d["value_cache"], d["block_tables"],
                                      d["context_lens"], step["scale"], partition_tokens=-1)
     assert (out[qs[1:].long().cuda() - 1].float() - dec.float()).abs().max().item() <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+def test_prefill_growing_scores(dtype):
+    """Keys grow along the context, so each row's running maximum keeps
+    moving by more than 2^8 in weight: every rescale of the running output
+    is exercised, and the result must still be the one-pass softmax.  The
+    attention is then nearly one-hot, so outputs take the size of single V
+    entries; V is scaled by 1/4 to keep them below 2, where rounding the
+    output to the storage type stays inside the fixed absolute bound."""
+    lens, chunks = [900, 333], [600, 333]
+    step, q, qs = _case(lens, chunks, 8, 2, 128, 16, dtype, seed=5)
+    kc = step["key_cache"].float()
+    tables = step["block_tables"]
+    for s_, L in enumerate(lens):
+        for k in range((L + 15) // 16):
+            kc[int(tables[s_, k])] *= 1.0 + 0.25 * k
+    step["key_cache"] = kc.to(_DT[dtype])
+    step["value_cache"] = (step["value_cache"].float() * 0.25).to(_DT[dtype])
+    q = (q.float() * 2.0).to(_DT[dtype])
+    _check(step, q, qs, chunks)
