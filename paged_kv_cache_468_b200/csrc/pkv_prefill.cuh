@@ -13,17 +13,20 @@
 // located through the block table, exactly as the decode kernels do):
 //
 //   S_j  = Q K_j^T        tcgen05.mma, Q and K_j in shared memory, S in TMEM
-//   P_j  = 2^(S_j*scale*log2e - m)    one row per softmax thread, bf16/f16
-//                                      into shared memory
-//   O   += P_j V_j         tcgen05.mma, O in TMEM (V read MN-major)
+//   P_j  = 2^(S_j*scale*log2e - m)    one row per softmax thread, bf16/f16,
+//                                      stored over S_j in TMEM
+//   O   += P_j V_j         tcgen05.mma, P from TMEM, V from shared memory
+//                          (read MN-major), O in TMEM
 //
 // The running row maximum m is only moved when a tile's maximum exceeds it
 // by more than 2^8 (P then stays <= 256); O and the row sum are rescaled by
 // the softmax warps at that point, so the result equals the one-pass softmax
-// up to rounding.  Warp roles: 0-3 softmax + epilogue (warp w owns TMEM lanes
-// 32w..32w+31), 4 loads Q and the K ring, 5 allocates TMEM and issues every
-// MMA, 6 loads the V ring and clears V rows past the last visible key (so
-// masked weights meet finite values).  Every wait is bounded; on a time-out
+// up to rounding.  S (and P over it) is double-buffered in TMEM: the
+// softmax of tile j+1 reads its scores while P_j V_j runs.
+// Warp roles: 0-3 softmax + epilogue (warp w owns TMEM lanes 32w..32w+31),
+// 4 loads Q and the K ring (3 stages), 5 allocates TMEM and issues every MMA,
+// 6 loads the V ring (2 stages) and clears V rows past the last visible key
+// (so masked weights meet finite values).  Every wait is bounded; on a time-out
 // the CTA records PKV_DEVFLAG_WAIT_TIMEOUT, lets in-flight copies and MMAs
 // finish and frees its TMEM.
 #pragma once
@@ -52,7 +55,9 @@ struct PrefillArgs {
 constexpr int kPfRows = 128;             // query rows per CTA (MMA M)
 constexpr int kPfKeys = 64;              // keys per tile (N of Q K^T, K of P V)
 constexpr int kPfThreads = 224;          // 7 warps
-constexpr uint32_t kPfTmemCols = 256;    // S: 2 x 64 columns, O: D columns at 128
+constexpr uint32_t kPfTmemCols = 256;    // S/P: 2 x 64 columns, O: D columns at 128
+constexpr int kPfKStages = 3;
+constexpr int kPfVStages = 2;
 
 template <int D>
 struct PfShape {
@@ -61,32 +66,35 @@ struct PfShape {
     static constexpr int kKVHalf = kPfKeys * 128;           // one half of a K or V tile
     static constexpr int kQBytes = kHalves * kQHalf;
     static constexpr int kKVBytes = kHalves * kKVHalf;
-    static constexpr int kPBytes = kPfRows * kPfKeys * 2;   // 128 rows x 128 B
     static constexpr int kQOff = 0;
-    static constexpr int kKOff = kQOff + kQBytes;           // 2 stages
-    static constexpr int kVOff = kKOff + 2 * kKVBytes;      // 2 stages
-    static constexpr int kPOff = kVOff + 2 * kKVBytes;
-    static constexpr int kDataBytes = kPOff + kPBytes;
+    static constexpr int kKOff = kQOff + kQBytes;
+    static constexpr int kVOff = kKOff + kPfKStages * kKVBytes;
+    static constexpr int kDataBytes = kVOff + kPfVStages * kKVBytes;
     // + 1024 so that the data can start on a 1024-byte boundary; the barriers
     // sit in whichever end of that slack has room
-    static constexpr int kSmemBytes = kDataBytes + 1024;
+    // two CTAs per SM, never three: a third would wait for TMEM (2 x 256
+    // columns fill the SM's 512) instead of working
+    static constexpr int kSmemBytes = (kDataBytes + 1024 > 80 * 1024) ? kDataBytes + 1024 : 80 * 1024;
 };
 
 // mbarrier slots
 enum PfBar {
     kBarQFull = 0,
-    kBarKFull = 1,     // 2
-    kBarKEmpty = 3,    // 2
-    kBarVFull = 5,     // 2
-    kBarVEmpty = 7,    // 2
-    kBarSFull = 9,     // 2
-    kBarPFull = 11,
-    kBarODone = 12,
-    kBarVTail = 13,
-    kBarDrain = 14,
-    kBarTmemSlot = 15,   // not a barrier: the TMEM base address
-    kNumPfBars = 16
+    kBarKFull = 1,     // kPfKStages
+    kBarKEmpty = 4,    // kPfKStages
+    kBarVFull = 7,     // kPfVStages
+    kBarVEmpty = 9,    // kPfVStages
+    kBarSFull = 11,    // 2, one per S/P buffer
+    kBarPFull = 13,    // 2, one per S/P buffer
+    kBarODone = 15,
+    kBarVTail = 16,
+    kBarDrain = 17,
+    kBarTmemSlot = 18,   // not a barrier: the TMEM base address
+    kNumPfBars = 20
 };
+// A barrier per S/P buffer completes once per two tiles, and buffer j & 1 is
+// refilled (S_{j+2}) only after the MMA thread consumed P_j: no barrier can
+// run two phases ahead of its waiter.
 
 template <int D, int BS, bool BF16>
 __global__ void __launch_bounds__(kPfThreads, 2)
@@ -100,6 +108,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     constexpr int KS = D / 16;               // k-steps of Q K^T
     constexpr int KV_STEPS = kPfKeys / 16;   // k-steps of P V
     constexpr int BPT = kPfKeys / BS;        // cache blocks per key tile
+    static_assert(32 % BPT == 0, "a key tile's block ids lie in one 32-id window");
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const uint32_t raw_s = smem_addr(smem_raw);
@@ -121,14 +130,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQFull), 1);
 #pragma unroll
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < kPfKStages; ++s) {
             mbar_init(bar(kBarKFull + s), 1);
             mbar_init(bar(kBarKEmpty + s), 1);
+        }
+#pragma unroll
+        for (int s = 0; s < kPfVStages; ++s) {
             mbar_init(bar(kBarVFull + s), 1);
             mbar_init(bar(kBarVEmpty + s), 1);
-            mbar_init(bar(kBarSFull + s), 1);
         }
-        mbar_init(bar(kBarPFull), 128);
+        mbar_init(bar(kBarSFull + 0), 1);
+        mbar_init(bar(kBarSFull + 1), 1);
+        mbar_init(bar(kBarPFull + 0), 4);       // one arrive per softmax warp
+        mbar_init(bar(kBarPFull + 1), 4);
         mbar_init(bar(kBarODone), 1);
         mbar_init(bar(kBarVTail), 1);
         mbar_init(bar(kBarDrain), 1);
@@ -179,7 +193,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t sQ = data_s + Sh::kQOff;
     const uint32_t sK = data_s + Sh::kKOff;
     const uint32_t sV = data_s + Sh::kVOff;
-    const uint32_t sP = data_s + Sh::kPOff;
 
     if (warp == 4 || warp == 6) {
         // ---- loads: warp 4 Q and the K ring, warp 6 the V ring ----
@@ -188,48 +201,61 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const int full0 = is_k ? kBarKFull : kBarVFull;
         const int empty0 = is_k ? kBarKEmpty : kBarVEmpty;
         const uint32_t ring = is_k ? sK : sV;
+        const int NS = is_k ? kPfKStages : kPfVStages;
         int issued = 0;
-        if (lane == 0) {
+        {
+            // the whole warp walks the tiles: block ids are read 32 at a time,
+            // one per lane, and lane 0 issues the copies
             const uint64_t policy = policy_evict_normal();   // the sequence's other CTAs reread them
             const int32_t *trow = a.block_tables + (size_t)b * a.max_blocks;
-            if (is_k) {
+            if (is_k && lane == 0) {
                 mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(Sh::kHalves * R * 128));
 #pragma unroll
                 for (int h = 0; h < Sh::kHalves; ++h)
                     tma_load_3d(sQ + h * Sh::kQHalf, &tm_q, bar(kBarQFull), h * 64, kvh * G, q0 + i0,
                                 policy);
             }
+            int ids = 0;
             for (int j = 0; j < nt; ++j) {
-                const int s = j & 1;
-                if (j >= 2 &&
-                    !mbar_wait_bounded(bar(empty0 + s), (uint32_t)(((j >> 1) - 1) & 1), kWaitLimitNs)) {
-                    raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-                    break;
-                }
-                const int kb0 = j * BPT;
-                const int nb = min(BPT, nblk - kb0);
-                mbar_arrive_expect_tx(bar(full0 + s), (uint32_t)(nb * BS * D * 2));
-                for (int i = 0; i < nb; ++i) {
-                    int blk = __ldg(trow + kb0 + i);
-                    if ((unsigned)blk >= (unsigned)a.num_blocks) {
-                        raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
-                        blk = 0;
+                const int s = j % NS;
+                if (j >= NS) {
+                    const bool free_ =
+                        mbar_wait_bounded(bar(empty0 + s), (uint32_t)((j / NS - 1) & 1), kWaitLimitNs);
+                    if (!__all_sync(0xffffffffu, free_)) {
+                        if (lane == 0)
+                            raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+                        break;
                     }
+                }
+                const int kb0 = j * BPT;                   // a tile never straddles 32 ids
+                const int nb = min(BPT, nblk - kb0);
+                if ((kb0 & 31) == 0)
+                    ids = kb0 + lane < nblk ? __ldg(trow + kb0 + lane) : 0;
+                if (lane == 0)
+                    mbar_arrive_expect_tx(bar(full0 + s), (uint32_t)(nb * BS * D * 2));
+                for (int i = 0; i < nb; ++i) {
+                    int blk = __shfl_sync(0xffffffffu, ids, (kb0 + i) & 31);
+                    if (lane == 0) {
+                        if ((unsigned)blk >= (unsigned)a.num_blocks) {
+                            raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
+                            blk = 0;
+                        }
 #pragma unroll
-                    for (int h = 0; h < Sh::kHalves; ++h)
-                        tma_load_3d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
-                                    bar(full0 + s), h * 64, kvh, blk * BS, policy);
+                        for (int h = 0; h < Sh::kHalves; ++h)
+                            tma_load_3d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
+                                        bar(full0 + s), h * 64, kvh, blk * BS, policy);
+                    }
                 }
                 issued = j + 1;
             }
         }
-        issued = __shfl_sync(0xffffffffu, issued, 0);
         if (!is_k && issued == nt) {
             // V rows of the last tile past p_max (the context's tail in its last
             // block, and blocks never loaded) are cleared once the tile landed
             const int j = nt - 1;
-            const int s = j & 1;
-            const bool landed = mbar_wait_bounded(bar(kBarVFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
+            const int s = j % kPfVStages;
+            const bool landed =
+                mbar_wait_bounded(bar(kBarVFull + s), (uint32_t)((j / kPfVStages) & 1), kWaitLimitNs);
             if (__all_sync(0xffffffffu, landed)) {
                 const int z0 = p_max + 1 - j * kPfKeys;   // first row to clear, 1 .. 64
                 if (z0 < kPfKeys) {
@@ -254,55 +280,67 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (lane == 0) {
             if (is_k)
                 mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs / 8);
-            for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j)
-                mbar_wait_bounded(bar(full0 + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs / 8);
+            for (int j = issued > NS ? issued - NS : 0; j < issued; ++j)
+                mbar_wait_bounded(bar(full0 + j % NS), (uint32_t)((j / NS) & 1), kWaitLimitNs / 8);
         }
     } else if (warp == 5) {
         // ---- MMA issue: one thread ----
         if (lane == 0) {
             constexpr uint32_t idS = f16_idesc<BF16>(kPfRows, kPfKeys, false);
             constexpr uint32_t idO = f16_idesc<BF16>(kPfRows, D, true);
-            // S_j = Q K_j^T into S buffer j & 1; Q and K K-major, 128-byte rows
+            // S_j = Q K_j^T into S buffer j & 1; Q and K K-major, 128-byte rows.
+            // Buffer j & 1 last held P_{j-2}, read by P_{j-2} V_{j-2}: MMAs into
+            // different accumulators are not ordered with each other, so the
+            // caller waits for that MMA to complete first.
             auto issue_s = [&](int j) -> bool {
-                const int s = j & 1;
-                if (!mbar_wait_bounded(bar(kBarKFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs))
+                const int ks_ = j % kPfKStages;
+                if (!mbar_wait_bounded(bar(kBarKFull + ks_), (uint32_t)((j / kPfKStages) & 1),
+                                       kWaitLimitNs))
                     return false;
                 tc_fence_after();
-                const uint32_t kt = sK + s * Sh::kKVBytes;
+                const uint32_t kt = sK + ks_ * Sh::kKVBytes;
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
                     const uint32_t koff = (uint32_t)((ks & 3) * 32);   // 16 elements = 32 bytes
-                    tc_mma_f16(tmem + s * kPfKeys,
+                    tc_mma_f16(tmem + (j & 1) * kPfKeys,
                                sw128_desc(sQ + (ks >> 2) * Sh::kQHalf + koff, 16, 1024),
                                sw128_desc(kt + (ks >> 2) * Sh::kKVHalf + koff, 16, 1024), idS,
                                ks > 0 ? 1u : 0u);
                 }
-                tc_commit(bar(kBarSFull + s));
-                tc_commit(bar(kBarKEmpty + s));
+                tc_commit(bar(kBarSFull + (j & 1)));
+                tc_commit(bar(kBarKEmpty + ks_));
                 return true;
             };
             bool ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
             for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt && !(ok = issue_s(j + 1)))
-                    break;
-                const int s = j & 1;
-                ok = mbar_wait_bounded(bar(kBarPFull), (uint32_t)(j & 1), kWaitLimitNs) &&
-                     mbar_wait_bounded(bar(kBarVFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
+                if (j + 1 < nt) {
+                    // P_{j-1} V_{j-1} reads buffer (j+1) & 1; O_DONE is at most one
+                    // phase past j-1 here (P_j V_j is not issued yet)
+                    if (j >= 1 &&
+                        !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs)))
+                        break;
+                    if (!(ok = issue_s(j + 1)))
+                        break;
+                }
+                const int vs = j % kPfVStages;
+                ok = mbar_wait_bounded(bar(kBarPFull + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
+                     mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((j / kPfVStages) & 1),
+                                       kWaitLimitNs) &&
                      (j + 1 < nt || mbar_wait_bounded(bar(kBarVTail), 0u, kWaitLimitNs));
                 if (!ok)
                     break;
                 tc_fence_after();
-                // O += P_j V_j: P K-major (keys along its 128-byte rows), V
-                // MN-major (head dim along the rows: halves LBO apart, 8-key
-                // groups 1024 bytes apart)
-                const uint32_t vt = sV + s * Sh::kKVBytes;
+                // O += P_j V_j: P from TMEM (16 keys = 8 packed columns per
+                // k-step), V MN-major (head dim along the rows: halves LBO
+                // apart, 8-key groups 1024 bytes apart)
+                const uint32_t vt = sV + vs * Sh::kKVBytes;
+                const uint32_t tp = tmem + (j & 1) * kPfKeys;
 #pragma unroll
                 for (int kk = 0; kk < KV_STEPS; ++kk)
-                    tc_mma_f16(tO, sw128_desc(sP + kk * 32, 16, 1024),
-                               sw128_desc(vt + kk * 16 * 128, Sh::kKVHalf, 1024), idO,
-                               (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_mma_f16_ts(tO, tp + kk * 8, sw128_desc(vt + kk * 16 * 128, Sh::kKVHalf, 1024),
+                                  idO, (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(bar(kBarODone));
-                tc_commit(bar(kBarVEmpty + s));
+                tc_commit(bar(kBarVEmpty + vs));
             }
             if (!ok)
                 raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
@@ -320,7 +358,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         float m_used = kNegInf;
         float l = 0.f;
         bool ok = true;
-        uint8_t *prow = data + Sh::kPOff + r * 128;
+        // for a positive scale the maximum is taken on the raw scores and the
+        // scale is folded into the exponent, p = 2^(s*scale - m)
+        const float sc = a.scale_log2;
+        const bool fold = sc > 0.f;
+        const float sm = fold ? 1.f : sc;       // applied before the maximum
+        const float se = fold ? sc : 1.f;       // applied in the exponent
         for (int j = 0; j < nt; ++j) {
             const int s = j & 1;
             ok = mbar_wait_bounded(bar(kBarSFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
@@ -331,22 +374,29 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             tc_fence_after();
             uint32_t raw[64];
             tmem_ld64(tmem + lane_base + s * kPfKeys, raw);
+            // eight independent max / sum chains, not 64-long ones
             float x[64];
-            float mt = kNegInf;
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mx[i] = kNegInf;
             const int t0 = j * kPfKeys;
             if (t0 + kPfKeys - 1 <= pos0) {         // every key visible to every row
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
-                    x[c] = __uint_as_float(raw[c]) * a.scale_log2;
-                    mt = fmaxf(mt, x[c]);
+                    x[c] = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
+                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
             } else {
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
-                    x[c] = t0 + c <= pos ? __uint_as_float(raw[c]) * a.scale_log2 : kNegInf;
-                    mt = fmaxf(mt, x[c]);
+                    const float v = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
+                    x[c] = t0 + c <= pos ? v : kNegInf;
+                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
             }
+            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * se;
             const bool resc = mt > m_used + 8.f;    // first tile: m_used = -inf
             const float m_new = resc ? mt : m_used;
             const float alpha = resc ? ex2(m_used - m_new) : 1.f;
@@ -354,45 +404,51 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
             // the row sum is taken over the rounded weights the MMA multiplies,
             // so the normalised weights sum to one exactly
             uint32_t pk[32];
-            float rs = 0.f;
+            float rsv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                rsv[i] = 0.f;
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                pk[c] = pack2<BF16>(ex2(x[2 * c] - msub), ex2(x[2 * c + 1] - msub));
+                pk[c] = pack2<BF16>(ex2(fmaf(x[2 * c], se, -msub)), ex2(fmaf(x[2 * c + 1], se, -msub)));
                 const float2 pr = unpack2<BF16>(pk[c]);
-                rs += pr.x + pr.y;
+                rsv[c & 7] += pr.x + pr.y;
             }
+            const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
             l = l * alpha + rs;
             m_used = m_new;
             if (j > 0) {
-                // the P buffer and O belong to P_{j-1} V_{j-1} until it completes
+                // P_j is stored only once P_{j-1} V_{j-1} has completed (O then
+                // holds it, for a rescale).  Storing P_j into TMEM while that MMA
+                // was still running gave intermittently wrong rows on B200 (10-40%
+                // of runs of a 7-token chunk over 520 keys); with the wait, none in
+                // hundreds of runs.  O_DONE is at most one phase ahead of this
+                // wait: P_j V_j needs this warp's P_j.
                 ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, resc)) {
+            }
+            if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t o[32];
-                        tmem_ld32(tO + lane_base + c0, o);
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + lane_base + c0, o);
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
-                            o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tmem_st32(tO + lane_base + c0, o);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + lane_base + c0, o);
                 }
             }
-            // P row r into the 128-byte swizzled layout: 16-byte chunk c of the
-            // row goes to chunk c ^ (r & 7)
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-                *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) =
-                    make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-            fence_proxy_async_smem();
+            // P_j over the first 32 columns of S_j (already read into registers)
+            tmem_st32(tmem + lane_base + s * kPfKeys, pk);
+            tmem_wait_st();
             tc_fence_before();
-            mbar_arrive(bar(kBarPFull));
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(kBarPFull + s));
         }
         if (ok)
             ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((nt - 1) & 1), kWaitLimitNs);
