@@ -460,7 +460,7 @@ def run_gpu(args, cfg, world, rank, local):
                 "traffic": committed_traffic(cfg.name),
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6650 GB/s",
-                "kernel": ("prefix_decode_kernel + paged_decode_kernel (suffixes) + "
+                "kernel": ("prefix_tc_kernel + paged_decode_kernel (suffixes) + "
                            "lse_merge_cascade_kernel" if cascade else
                            "paged_decode_kernel" + (" + lse_merge_kernel" if plan_np > 1 else "")),
                 "bytes_per_launch": nbytes["decode_unique"], "launch_ms": round(decode_ms, 5),

@@ -522,8 +522,7 @@ struct CascadePlan {
     int pt;        // partition length in tokens (prefix and suffix)
     int pp;        // prefix partitions
     int ps;        // suffix partitions
-    int nwq;       // consumer warps per prefix CTA
-    int chunks;    // member chunks per group
+    int chunks;    // member chunks per group (128 query rows per prefix CTA)
     size_t m_p, l_p, o_p, m_s, l_s, o_s, total;   // workspace offsets
 };
 
@@ -542,9 +541,8 @@ pkv_status cascade_plan(int batch, int Hq, int Hkv, int D, int max_prefix_blocks
     c->pt = partition_tokens > 0 ? (partition_tokens + bs - 1) / bs * bs : kAutoPartitionTokens;
     c->pp = (max_prefix_blocks * bs + c->pt - 1) / c->pt;
     c->ps = (max_suffix_blocks * bs + c->pt - 1) / c->pt;
-    const int rows = max_group_size * (Hq / Hkv);
-    c->nwq = rows <= 8 ? 1 : (rows <= 16 ? 2 : (rows <= 32 ? 4 : 8));
-    c->chunks = (rows + c->nwq * 8 - 1) / (c->nwq * 8);
+    const int members_per_cta = pkv::kPfRows / (Hq / Hkv);
+    c->chunks = (max_group_size + members_per_cta - 1) / members_per_cta;
     const size_t rp = (size_t)batch * Hq * c->pp, rs = (size_t)batch * Hq * c->ps;
     c->m_p = 0;
     c->l_p = align256(c->m_p + rp * 4);
@@ -556,42 +554,31 @@ pkv_status cascade_plan(int batch, int Hq, int Hkv, int D, int max_prefix_blocks
     return PKV_OK;
 }
 
-template <int D, int BS, bool BF16, int NWQ>
-cudaError_t launch_prefix(const CUtensorMap &mk, const CUtensorMap &mv, const pkv::CascadeArgs &c,
-                          cudaStream_t st)
+template <int D, int BS, bool BF16>
+cudaError_t launch_prefix(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                          const pkv::CascadeArgs &c, cudaStream_t st)
 {
-    constexpr int S = BS == 16 ? 4 : 3;
-    using Shape = pkv::DecodeShape<D, BS, 1, S>;
-    constexpr int smem = S * Shape::kStageBytes + 1024;
-    auto kern = pkv::prefix_decode_kernel<D, BS, BF16, NWQ, S>;
+    constexpr int smem = pkv::PfShape<D>::kSmemBytes;
+    auto kern = pkv::prefix_tc_kernel<D, BS, BF16>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)   // two CTAs (and their TMEM) per SM
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess)
         return e;
     const dim3 grid((unsigned)c.num_parts, (unsigned)c.num_kv_heads,
                     (unsigned)((size_t)c.num_groups * c.chunks));
-    return launch_pdl(kern, grid, dim3((NWQ + 1) * 32), smem, st, mk, mv, c);
-}
-
-template <int D, int BS, bool BF16>
-cudaError_t dispatch_prefix_nwq(int nwq, const CUtensorMap &mk, const CUtensorMap &mv,
-                                const pkv::CascadeArgs &c, cudaStream_t st)
-{
-    switch (nwq) {
-    case 1: return launch_prefix<D, BS, BF16, 1>(mk, mv, c, st);
-    case 2: return launch_prefix<D, BS, BF16, 2>(mk, mv, c, st);
-    case 4: return launch_prefix<D, BS, BF16, 4>(mk, mv, c, st);
-    default: return launch_prefix<D, BS, BF16, 8>(mk, mv, c, st);
-    }
+    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, mk, mv, c);
 }
 
 template <bool BF16>
-cudaError_t dispatch_prefix(int D, int bs, int nwq, const CUtensorMap &mk, const CUtensorMap &mv,
-                            const pkv::CascadeArgs &c, cudaStream_t st)
+cudaError_t dispatch_prefix(int D, int bs, const CUtensorMap &mq, const CUtensorMap &mk,
+                            const CUtensorMap &mv, const pkv::CascadeArgs &c, cudaStream_t st)
 {
-    if (D == 64 && bs == 16) return dispatch_prefix_nwq<64, 16, BF16>(nwq, mk, mv, c, st);
-    if (D == 64 && bs == 32) return dispatch_prefix_nwq<64, 32, BF16>(nwq, mk, mv, c, st);
-    if (D == 128 && bs == 16) return dispatch_prefix_nwq<128, 16, BF16>(nwq, mk, mv, c, st);
-    return dispatch_prefix_nwq<128, 32, BF16>(nwq, mk, mv, c, st);
+    if (D == 64 && bs == 16) return launch_prefix<64, 16, BF16>(mq, mk, mv, c, st);
+    if (D == 64 && bs == 32) return launch_prefix<64, 32, BF16>(mq, mk, mv, c, st);
+    if (D == 128 && bs == 16) return launch_prefix<128, 16, BF16>(mq, mk, mv, c, st);
+    return launch_prefix<128, 32, BF16>(mq, mk, mv, c, st);
 }
 
 }  // namespace
@@ -675,10 +662,16 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     c.scale_log2 = scale_log2;
     cudaError_t e = cudaSuccess;
     if (num_groups > 0) {
-        e = dtype == PKV_BF16 ? dispatch_prefix<true>(head_dim, block_size, plan.nwq, mk, mv, c, st)
-                              : dispatch_prefix<false>(head_dim, block_size, plan.nwq, mk, mv, c, st);
+        // the members of a group are consecutive query rows: a Q tile is
+        // 128/G members x the G heads of one kv head
+        CUtensorMap mq;
+        if ((s = make_query_map(&mq, query, batch, num_heads, head_dim, c.group,
+                                pkv::kPfRows / c.group, dtype)) != PKV_OK)
+            return s;
+        e = dtype == PKV_BF16 ? dispatch_prefix<true>(head_dim, block_size, mq, mk, mv, c, st)
+                              : dispatch_prefix<false>(head_dim, block_size, mq, mk, mv, c, st);
         if (e != cudaSuccess)
-            return cuda_fail(e, "prefix_decode_kernel launch");
+            return cuda_fail(e, "prefix_tc_kernel launch");
     }
 
     // level 2: each sequence's own blocks, as partition records

@@ -535,16 +535,14 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // Parallel samples of one prompt share the prompt's blocks ("23.1 vLLM：高吞吐
 // 推理框架原理与部署", section 二.3).  Sequences group_start[g] ..
 // group_start[g+1]-1 share the prefix_lens[g] tokens (a multiple of the block
-// size) listed in prefix_tables[g].  One CTA per (prefix partition, kv head,
-// group member chunk): a producer warp streams the partition's K/V blocks
-// through a CTA-wide ring of S stages (TMA, full/empty mbarriers), and each
-// of NWQ consumer warps applies 8 of the group's query rows (member, head of
-// the GQA group) to every tile, so each prefix block is read from HBM once per
-// group instead of once per sequence.  Each consumer writes, per query row,
-// the partition's record (max, normaliser, normalised row); level 2 (the
-// decode kernel over each sequence's own suffix, records only) and the
-// cascade merge complete the result, which equals the decode over the
-// concatenated table.
+// size) listed in prefix_tables[g].  Level 1 (prefix_tc_kernel, in
+// pkv_prefill.cuh) runs one CTA per (prefix partition, kv head, chunk of
+// 128 / G members) on the tensor cores, so each prefix block is read from HBM
+// once per group instead of once per sequence, and writes per query row the
+// partition's record (max, normaliser, normalised row); level 2 (the decode
+// kernel over each sequence's own suffix, records only) and the cascade merge
+// below complete the result, which equals the decode over the concatenated
+// table.
 struct CascadeArgs {
     const uint16_t *query;           // [B, Hq, D]
     const int32_t *prefix_tables;    // [num_groups, max_prefix_blocks]
@@ -566,194 +564,6 @@ struct CascadeArgs {
     int chunks;                      // member chunks per group
     float scale_log2;
 };
-
-template <int D, int BS, bool BF16, int NWQ, int S>
-// Up to 4 consumer warps the kernel is held to 128 registers so that three
-// CTAs share an SM: the consumers are latency-bound (mma, shuffles, waits)
-// and need the extra warps; 8-warp CTAs would spill at that limit.
-__global__ void __launch_bounds__((NWQ + 1) * 32, (NWQ <= 4 ? 3 : 1))
-prefix_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                     const CascadeArgs a)
-{
-    using Shape = DecodeShape<D, BS, 1, S>;
-    constexpr int kHalfBytes = Shape::kHalfBytes;
-    constexpr int kTileBytes = Shape::kTileBytes;
-    constexpr int kStageBytes = Shape::kStageBytes;
-    constexpr int KS = D / 16;
-
-    extern __shared__ uint8_t smem_raw[];
-    __shared__ __align__(8) uint64_t full[S];
-    __shared__ __align__(8) uint64_t empty[S];
-    uint8_t *smem = reinterpret_cast<uint8_t *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const uint32_t ring_s = smem_addr(smem);
-
-    const int pp = blockIdx.x;
-    const int kvh = blockIdx.y;
-    const int g = blockIdx.z / a.chunks;
-    const int mc = blockIdx.z - g * a.chunks;
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int G = a.group;
-
-    if (threadIdx.x == 0) {
-#pragma unroll
-        for (int s = 0; s < S; ++s) {
-            mbar_init(smem_addr(&full[s]), 1);
-            mbar_init(smem_addr(&empty[s]), NWQ);
-        }
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
-    }
-    fence_mbar_init();
-    __syncthreads();
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("griddepcontrol.launch_dependents;");
-
-    int first = __ldg(a.group_start + g);
-    int count = __ldg(a.group_start + g + 1) - first;
-    if (first < 0 || count < 0 || first + count > a.batch || count > a.max_group_size) {
-        if (threadIdx.x == 0 && pp == 0 && kvh == 0 && mc == 0)
-            raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
-        first = first < 0 ? 0 : (first > a.batch ? a.batch : first);
-        count = count < 0 ? 0 : count;
-        count = min(count, min(a.max_group_size, a.batch - first));
-    }
-    const int row0 = mc * NWQ * 8;                  // first query row of this chunk
-    const int nrows = min(NWQ * 8, count * G - row0);
-    int Lp = __ldg(a.prefix_lens + g);
-    const int span = a.max_prefix_blocks * BS;
-    if (Lp < 0 || Lp > span || Lp % BS != 0) {
-        if (threadIdx.x == 0 && pp == 0 && kvh == 0 && mc == 0)
-            raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
-        Lp = Lp < 0 ? 0 : (Lp > span ? span : Lp - Lp % BS);
-    }
-    const int tok0 = pp * a.part_tokens;
-    const int tok1 = min(Lp, tok0 + a.part_tokens);
-    if (nrows <= 0 || tok1 <= tok0)
-        return;                                     // nothing here (the merge skips it)
-    const int nblk = (tok1 - tok0) / BS;
-    const int blk0 = tok0 / BS;
-
-    if (warp == NWQ) {
-        // ---- producer: one block per stage, S ahead of the consumers ----
-        const int32_t *trow = a.prefix_tables + (size_t)g * a.max_prefix_blocks + blk0;
-        const uint64_t policy = policy_evict_first();
-        int ids = 0;
-        for (int k = 0; k < nblk; ++k) {
-            const int s = k % S;
-            if (k >= S) {
-                const bool ok = mbar_wait_bounded(smem_addr(&empty[s]), (uint32_t)(((k / S) - 1) & 1),
-                                                  kWaitLimitNs);
-                if (!__all_sync(0xffffffffu, ok)) {
-                    if (lane == 0)
-                        raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-                    break;
-                }
-            }
-            if ((k & 31) == 0)
-                ids = k + lane < nblk ? __ldg(trow + k + lane) : 0;
-            int blk = __shfl_sync(0xffffffffu, ids, k & 31);
-            if ((unsigned)blk >= (unsigned)a.num_blocks) {
-                if (lane == 0)
-                    raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
-                blk = 0;
-            }
-            if (lane == 0) {
-                const uint32_t bar = smem_addr(&full[s]);
-                const uint32_t dk = ring_s + (uint32_t)(s * kStageBytes);
-                mbar_arrive_expect_tx(bar, kStageBytes);
-#pragma unroll
-                for (int h = 0; h < Shape::kHalves; ++h) {
-                    tma_load_3d(dk + h * kHalfBytes, &tm_k, bar, h * 64, kvh, blk * BS, policy);
-                    tma_load_3d(dk + kTileBytes + h * kHalfBytes, &tm_v, bar, h * 64, kvh, blk * BS,
-                                policy);
-                }
-            }
-        }
-        return;
-    }
-
-    // ---- consumers: warp w owns query rows row0 + 8w + n, n = 0..7 ----
-    uint32_t qf[KS][2];
-    const int n_own = lane >> 2;
-    const int r_own = row0 + warp * 8 + n_own;       // query row of column n_own
-    const bool col_ok = r_own < row0 + nrows;
-    {
-        const int member = r_own / G;
-        const int gq = r_own - member * G;
-        const int c = lane & 3;
-        const uint32_t *q32 = reinterpret_cast<const uint32_t *>(
-            a.query + ((size_t)(first + (col_ok ? member : 0)) * a.num_heads + (size_t)kvh * G +
-                       (col_ok ? gq : 0)) * D);
-#pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-            qf[ks][0] = col_ok ? __ldg(q32 + ks * 8 + c) : 0u;
-            qf[ks][1] = col_ok ? __ldg(q32 + ks * 8 + 4 + c) : 0u;
-        }
-    }
-    float m_run[2] = {kNegInf, kNegInf};
-    float l_run[2] = {0.f, 0.f};
-    float acc_hi[KS][4], acc_lo[KS][4];
-#pragma unroll
-    for (int dt = 0; dt < KS; ++dt)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            acc_hi[dt][i] = 0.f;
-            acc_lo[dt][i] = 0.f;
-        }
-    int consumed = 0;
-    for (int k = 0; k < nblk; ++k) {
-        const int s = k % S;
-        const bool got = mbar_wait_bounded(smem_addr(&full[s]), (uint32_t)((k / S) & 1), kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, got)) {
-            if (lane == 0)
-                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-            break;
-        }
-        consumed = k + 1;
-        const uint32_t sk = ring_s + (uint32_t)(s * kStageBytes);
-        attend_block<D, BS, BF16>(sk, sk + kTileBytes, BS, qf, a.scale_log2, m_run, l_run, acc_hi,
-                                  acc_lo, lane);
-        __syncwarp();
-        if (lane == 0)
-            mbar_arrive(smem_addr(&empty[s]));      // this warp is done with the stage
-    }
-    // stages the producer filled but this warp did not consume (a wait gave up)
-    for (int k = consumed; k < nblk && k < consumed + S; ++k)
-        mbar_wait_bounded(smem_addr(&full[k % S]), (uint32_t)((k / S) & 1), kWaitLimitNs / 8);
-
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 4);
-        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 8);
-        l_run[j] += __shfl_xor_sync(0xffffffffu, l_run[j], 16);
-    }
-    // records of the lane's columns 2c, 2c+1
-    const int c = lane & 3;
-    const int r = lane >> 2;
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        const int n = 2 * c + j;
-        const int row_local = row0 + warp * 8 + n;
-        if (row_local >= row0 + nrows)
-            continue;
-        const int member = row_local / G;
-        const int gq = row_local - member * G;
-        const size_t row = (size_t)(first + member) * a.num_heads + (size_t)kvh * G + gq;
-        const size_t rec = row * a.num_parts + pp;
-        const float inv = l_run[j] > 0.f ? 1.f / l_run[j] : 0.f;
-#pragma unroll
-        for (int dt = 0; dt < KS; ++dt) {
-            a.rec_o[rec * D + dt * 16 + r] = (acc_hi[dt][j] + acc_lo[dt][j]) * inv;
-            a.rec_o[rec * D + dt * 16 + r + 8] = (acc_hi[dt][2 + j] + acc_lo[dt][2 + j]) * inv;
-        }
-        if (r == 0) {
-            a.rec_m[rec] = m_run[j];
-            a.rec_l[rec] = l_run[j];
-        }
-    }
-}
 
 // Cascade merge: row (b, h) = its group's prefix records (partitions of the
 // prefix) and its own suffix records (partitions of the suffix), folded by

@@ -1,5 +1,8 @@
-// pkv_prefill.cuh -- chunked prefill over the paged KV cache on the
-// 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory).
+// pkv_prefill.cuh -- many query rows over the paged KV cache on the
+// 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory):
+// chunked prefill (prefill_tc_kernel) and the shared-prefix pass of cascade
+// decode (prefix_tc_kernel, which differs only in its work map, no causal
+// mask, and its output: partition records for the cascade merge).
 //
 // Sequence b brings C_b = query_start[b+1] - query_start[b] new tokens, the
 // last C_b of its L_b = context_lens[b] cached tokens (their K/V were written
@@ -96,10 +99,14 @@ enum PfBar {
 // refilled (S_{j+2}) only after the MMA thread consumed P_j: no barrier can
 // run two phases ahead of its waiter.
 
-template <int D, int BS, bool BF16>
-__global__ void __launch_bounds__(kPfThreads, 2)
-prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a)
+// The body shared by the chunked prefill (PREFIX = false: causal rows of one
+// sequence's chunk) and the prefix pass of cascade decode (PREFIX = true: the
+// query rows of a group's members over one partition of their shared prefix,
+// written as partition records for the merge).
+template <int D, int BS, bool BF16, bool PREFIX>
+__device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
+                                          const CUtensorMap *tm_v, const PrefillArgs &a,
+                                          const CascadeArgs &c)
 {
     using Sh = PfShape<D>;
     static_assert(D == 64 || D == 128, "head_dim 64 or 128");
@@ -118,14 +125,15 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem_raw + (bars_s - raw_s));
     auto bar = [&](int i) { return bars_s + 8u * (uint32_t)i; };
 
-    const int tile = blockIdx.x;
     const int kvh = blockIdx.y;
-    const int b = blockIdx.z;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int G = a.group;
-    const int TT = kPfRows / G;   // query tokens per CTA
+    const int G = PREFIX ? c.group : a.group;
+    const int TT = kPfRows / G;   // query tokens (prefix: group members) per CTA
     const int R = TT * G;         // rows in use (128 when G divides 128)
+    const int num_heads = PREFIX ? c.num_heads : a.num_heads;
+    const int num_blocks = PREFIX ? c.num_blocks : a.num_blocks;
+    const float scale_log2 = PREFIX ? c.scale_log2 : a.scale_log2;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQFull), 1);
@@ -146,36 +154,79 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_init(bar(kBarODone), 1);
         mbar_init(bar(kBarVTail), 1);
         mbar_init(bar(kBarDrain), 1);
-        prefetch_tensormap(&tm_q);
-        prefetch_tensormap(&tm_k);
-        prefetch_tensormap(&tm_v);
+        prefetch_tensormap(tm_q);
+        prefetch_tensormap(tm_k);
+        prefetch_tensormap(tm_v);
     }
     fence_mbar_init();
     __syncthreads();
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
 
-    const int q0 = __ldg(a.query_start + b);
-    int C = __ldg(a.query_start + b + 1) - q0;
-    int L = __ldg(a.context_lens + b);
-    const int span = a.max_blocks * BS;
-    if (q0 < 0 || C < 0 || q0 + C > a.num_tokens || C > a.max_query_len || L < 0 || L > span ||
-        C > L) {
-        if (threadIdx.x == 0 && tile == 0 && kvh == 0)
-            raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
-        L = L < 0 ? 0 : (L > span ? span : L);
-        if (q0 < 0 || C < 0 || q0 + C > a.num_tokens)
-            C = 0;                                  // rows outside query/out: skip the sequence
-        C = min(C, min(L, a.max_query_len));
+    // The CTA's work: query rows row0 .. row0+127 of a row space of `rows`
+    // real rows ((token or member) x head of the group), whose first query
+    // row is query row q_tok0; keys 0 .. p_max of a key range that starts at
+    // block trow[0]; row r sees keys up to pos0 + r / G (prefill, causal) or
+    // all of them (prefix).
+    int rows, row0, q_tok0, p_max, pos0, rec_part = 0;
+    const int32_t *trow;
+    if constexpr (!PREFIX) {
+        const int tile = blockIdx.x;
+        const int b = blockIdx.z;
+        const int q0 = __ldg(a.query_start + b);
+        int C = __ldg(a.query_start + b + 1) - q0;
+        int L = __ldg(a.context_lens + b);
+        const int span = a.max_blocks * BS;
+        if (q0 < 0 || C < 0 || q0 + C > a.num_tokens || C > a.max_query_len || L < 0 || L > span ||
+            C > L) {
+            if (threadIdx.x == 0 && tile == 0 && kvh == 0)
+                raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+            L = L < 0 ? 0 : (L > span ? span : L);
+            if (q0 < 0 || C < 0 || q0 + C > a.num_tokens)
+                C = 0;                              // rows outside query/out: skip the sequence
+            C = min(C, min(L, a.max_query_len));
+        }
+        rows = C * G;
+        row0 = tile * R;
+        if (row0 >= rows)
+            return;                                 // whole CTA, before TMEM is touched
+        const int i0 = tile * TT;                   // first query token of the CTA
+        q_tok0 = q0 + i0;
+        pos0 = L - C + i0;                          // the first row's last key
+        p_max = L - C + min(C, i0 + TT) - 1;        // last key any row of the CTA sees
+        trow = a.block_tables + (size_t)b * a.max_blocks;
+    } else {
+        const int pp = blockIdx.x;
+        const int g = blockIdx.z / c.chunks;
+        const int mc = blockIdx.z - g * c.chunks;
+        int first = __ldg(c.group_start + g);
+        int count = __ldg(c.group_start + g + 1) - first;
+        if (first < 0 || count < 0 || first + count > c.batch || count > c.max_group_size) {
+            if (threadIdx.x == 0 && pp == 0 && kvh == 0 && mc == 0)
+                raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+            first = first < 0 ? 0 : (first > c.batch ? c.batch : first);
+            count = count < 0 ? 0 : count;
+            count = min(count, min(c.max_group_size, c.batch - first));
+        }
+        int Lp = __ldg(c.prefix_lens + g);
+        const int span = c.max_prefix_blocks * BS;
+        if (Lp < 0 || Lp > span || Lp % BS != 0) {
+            if (threadIdx.x == 0 && pp == 0 && kvh == 0 && mc == 0)
+                raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+            Lp = Lp < 0 ? 0 : (Lp > span ? span : Lp - Lp % BS);
+        }
+        const int tok0 = pp * c.part_tokens;
+        const int tok1 = min(Lp, tok0 + c.part_tokens);
+        rows = count * G;
+        row0 = mc * R;
+        if (row0 >= rows || tok1 <= tok0)
+            return;                                 // nothing here (the merge skips it)
+        q_tok0 = first + mc * TT;
+        p_max = tok1 - tok0 - 1;
+        pos0 = p_max;
+        trow = c.prefix_tables + (size_t)g * c.max_prefix_blocks + tok0 / BS;
+        rec_part = pp;
     }
-    const int rows = C * G;
-    const int row0 = tile * R;
-    if (row0 >= rows)
-        return;                                     // whole CTA, before TMEM is touched
-    const int i0 = tile * TT;                       // first query token of the CTA
-    const int last_tok = min(C, i0 + TT) - 1;
-    const int p_max = L - C + last_tok;             // last key any row of the CTA sees
-    const int pos0 = L - C + i0;                    // ... and the first row's last key
     const int nt = p_max / kPfKeys + 1;             // key tiles
     const int nblk = p_max / BS + 1;                // cache blocks read
 
@@ -197,7 +248,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (warp == 4 || warp == 6) {
         // ---- loads: warp 4 Q and the K ring, warp 6 the V ring ----
         const bool is_k = warp == 4;
-        const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+        const CUtensorMap *tm = is_k ? tm_k : tm_v;
         const int full0 = is_k ? kBarKFull : kBarVFull;
         const int empty0 = is_k ? kBarKEmpty : kBarVEmpty;
         const uint32_t ring = is_k ? sK : sV;
@@ -206,13 +257,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         {
             // the whole warp walks the tiles: block ids are read 32 at a time,
             // one per lane, and lane 0 issues the copies
-            const uint64_t policy = policy_evict_normal();   // the sequence's other CTAs reread them
-            const int32_t *trow = a.block_tables + (size_t)b * a.max_blocks;
+            // prefill: the sequence's other CTAs reread these blocks; prefix:
+            // each is read once per group and kv head
+            const uint64_t policy = PREFIX ? policy_evict_first() : policy_evict_normal();
             if (is_k && lane == 0) {
                 mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(Sh::kHalves * R * 128));
 #pragma unroll
                 for (int h = 0; h < Sh::kHalves; ++h)
-                    tma_load_3d(sQ + h * Sh::kQHalf, &tm_q, bar(kBarQFull), h * 64, kvh * G, q0 + i0,
+                    tma_load_3d(sQ + h * Sh::kQHalf, tm_q, bar(kBarQFull), h * 64, kvh * G, q_tok0,
                                 policy);
             }
             int ids = 0;
@@ -236,7 +288,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                 for (int i = 0; i < nb; ++i) {
                     int blk = __shfl_sync(0xffffffffu, ids, (kb0 + i) & 31);
                     if (lane == 0) {
-                        if ((unsigned)blk >= (unsigned)a.num_blocks) {
+                        if ((unsigned)blk >= (unsigned)num_blocks) {
                             raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
                             blk = 0;
                         }
@@ -354,13 +406,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const int grow = row0 + r;                  // row within the sequence
         const bool real = r < R && grow < rows;
-        const int pos = real ? L - C + grow / G : p_max;
+        const int pos = real && !PREFIX ? pos0 + r / G : p_max;
         float m_used = kNegInf;
         float l = 0.f;
         bool ok = true;
         // for a positive scale the maximum is taken on the raw scores and the
         // scale is folded into the exponent, p = 2^(s*scale - m)
-        const float sc = a.scale_log2;
+        const float sc = scale_log2;
         const bool fold = sc > 0.f;
         const float sm = fold ? 1.f : sc;       // applied before the maximum
         const float se = fold ? sc : 1.f;       // applied in the exponent
@@ -455,24 +507,46 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         if (__all_sync(0xffffffffu, ok)) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            const int i = real ? grow / G : 0;
-            const int g = real ? grow - i * G : 0;
-            uint4 *orow = reinterpret_cast<uint4 *>(
-                a.out + ((size_t)(q0 + i) * a.num_heads + (size_t)kvh * G + g) * D);
+            // query row (q_tok0 + r / G, head kvh * G + r % G): row0 is a multiple of G
+            const size_t orow_i = (size_t)(q_tok0 + r / G) * num_heads + (size_t)kvh * G + r % G;
+            if constexpr (!PREFIX) {
+                uint4 *orow = reinterpret_cast<uint4 *>(a.out + orow_i * D);
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
-                uint32_t o[32];
-                tmem_ld32(tO + lane_base + c0, o);
-                if (real) {
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + lane_base + c0, o);
+                    if (real) {
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        uint32_t w[4];
+                        for (int v = 0; v < 4; ++v) {
+                            uint32_t w[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            w[e] = pack2<BF16>(__uint_as_float(o[8 * v + 2 * e]) * inv,
-                                               __uint_as_float(o[8 * v + 2 * e + 1]) * inv);
-                        orow[c0 / 8 + v] = make_uint4(w[0], w[1], w[2], w[3]);
+                            for (int e = 0; e < 4; ++e)
+                                w[e] = pack2<BF16>(__uint_as_float(o[8 * v + 2 * e]) * inv,
+                                                   __uint_as_float(o[8 * v + 2 * e + 1]) * inv);
+                            orow[c0 / 8 + v] = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
                     }
+                }
+            } else {
+                // partition record: (m, l) with sum_k 2^(s_k) = 2^m * l, and O / l
+                const size_t rec = orow_i * c.num_parts + rec_part;
+                float4 *orec = reinterpret_cast<float4 *>(c.rec_o + rec * D);
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + lane_base + c0, o);
+                    if (real) {
+#pragma unroll
+                        for (int v = 0; v < 8; ++v)
+                            orec[c0 / 4 + v] = make_float4(__uint_as_float(o[4 * v]) * inv,
+                                                           __uint_as_float(o[4 * v + 1]) * inv,
+                                                           __uint_as_float(o[4 * v + 2]) * inv,
+                                                           __uint_as_float(o[4 * v + 3]) * inv);
+                    }
+                }
+                if (real) {
+                    c.rec_m[rec] = m_used;
+                    c.rec_l[rec] = l;
                 }
             }
         } else if (lane == 0) {
@@ -488,6 +562,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         tc_fence_after();
         tmem_dealloc(tmem, kPfTmemCols);
     }
+}
+
+template <int D, int BS, bool BF16>
+__global__ void __launch_bounds__(kPfThreads, 2)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a)
+{
+    tc_attend<D, BS, BF16, false>(&tm_q, &tm_k, &tm_v, a, CascadeArgs{});
+}
+
+template <int D, int BS, bool BF16>
+__global__ void __launch_bounds__(kPfThreads, 2)
+prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const CascadeArgs c)
+{
+    tc_attend<D, BS, BF16, true>(&tm_q, &tm_k, &tm_v, PrefillArgs{}, c);
 }
 
 }  // namespace pkv

@@ -117,7 +117,9 @@ def test_cascade_irregular_groups(D, bs, dtype):
         assert finite and err <= TOL[dtype], (pt, err, idx)
 
 
-@pytest.mark.parametrize("G,size", [(1, 8), (4, 8), (8, 16), (4, 32)])
+# a prefix CTA takes 128 query rows: 128/G members; the last three shapes
+# split a group over several CTAs (G = 3 leaves 2 rows of each CTA unused)
+@pytest.mark.parametrize("G,size", [(1, 8), (4, 8), (8, 16), (4, 32), (8, 40), (3, 50), (1, 130)])
 def test_cascade_group_shapes(G, size):
     Hkv = 2
     groups = [size, size]
