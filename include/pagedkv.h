@@ -249,10 +249,11 @@ pkv_status pkv_paged_attention_prefill(const void *query, int num_tokens, const 
  *
  * Sequence b attends over prefix_tables[g] (prefix_lens[g] tokens) followed by
  * suffix_tables[b] (suffix_lens[b] tokens); sequences outside every group
- * attend over their suffix only.  Three kernels: the prefix pass (a producer
- * warp streams each prefix block into a shared-memory ring, consumer warps
- * apply all of the group's query rows to it), the regular decode over the
- * suffixes writing partial records, and a log-sum-exp merge of both.
+ * attend over their suffix only.  Three kernels: the prefix pass (the
+ * group's query rows, 128 per CTA, against each 64-key tile of the prefix on
+ * the tcgen05 tensor cores, each prefix block read once per group), the
+ * regular decode over the suffixes writing partial records, and a
+ * log-sum-exp merge of both.
  * partition_tokens as for pkv_decode_plan (0: 512-token partitions).  Invalid
  * group bounds or prefix lengths set PKV_DEVFLAG_CONTEXT_RANGE.
  */
