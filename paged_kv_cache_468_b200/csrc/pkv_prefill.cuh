@@ -341,9 +341,8 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             constexpr uint32_t idS = f16_idesc<BF16>(kPfRows, kPfKeys, false);
             constexpr uint32_t idO = f16_idesc<BF16>(kPfRows, D, true);
             // S_j = Q K_j^T into S buffer j & 1; Q and K K-major, 128-byte rows.
-            // Buffer j & 1 last held P_{j-2}, read by P_{j-2} V_{j-2}: MMAs into
-            // different accumulators are not ordered with each other, so the
-            // caller waits for that MMA to complete first.
+            // Buffer j & 1 last held P_{j-2}, read by P_{j-2} V_{j-2}, issued
+            // earlier by this thread: its MMAs execute in issue order.
             auto issue_s = [&](int j) -> bool {
                 const int ks_ = j % kPfKStages;
                 if (!mbar_wait_bounded(bar(kBarKFull + ks_), (uint32_t)((j / kPfKStages) & 1),
@@ -365,15 +364,8 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             };
             bool ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
             for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt) {
-                    // P_{j-1} V_{j-1} reads buffer (j+1) & 1; O_DONE is at most one
-                    // phase past j-1 here (P_j V_j is not issued yet)
-                    if (j >= 1 &&
-                        !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs)))
-                        break;
-                    if (!(ok = issue_s(j + 1)))
-                        break;
-                }
+                if (j + 1 < nt && !(ok = issue_s(j + 1)))
+                    break;
                 const int vs = j % kPfVStages;
                 ok = mbar_wait_bounded(bar(kBarPFull + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
                      mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((j / kPfVStages) & 1),
@@ -470,12 +462,13 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             l = l * alpha + rs;
             m_used = m_new;
             if (j > 0) {
-                // P_j is stored only once P_{j-1} V_{j-1} has completed (O then
-                // holds it, for a rescale).  Storing P_j into TMEM while that MMA
-                // was still running gave intermittently wrong rows on B200 (10-40%
-                // of runs of a 7-token chunk over 520 keys); with the wait, none in
-                // hundreds of runs.  O_DONE is at most one phase ahead of this
-                // wait: P_j V_j needs this warp's P_j.
+                // P_j is stored only once P_{j-1} V_{j-1} has completed, so no
+                // MMA is running when TMEM is written (and O holds P_{j-1} V_{j-1}
+                // for a rescale).  Storing P_j while that MMA was still running
+                // gave intermittently wrong rows on B200 (10-40% of runs of a
+                // 7-token chunk over 520 keys); with the wait, none in hundreds
+                // of runs.  O_DONE is at most one phase ahead of this wait:
+                // P_j V_j needs this warp's P_j.
                 ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
