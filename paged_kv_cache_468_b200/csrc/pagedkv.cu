@@ -327,6 +327,8 @@ pkv_status pkv_copy_blocks(const void *src_key_cache, const void *src_value_cach
     if (block_bytes % 16 != 0)
         return fail(PKV_ERR_UNSUPPORTED, "block_bytes %lld is not a multiple of 16",
                     (long long)block_bytes);
+    if (num_pairs > (1 << 30))
+        return fail(PKV_ERR_UNSUPPORTED, "num_pairs %d > 2^30", num_pairs);
     if (num_pairs == 0)
         return PKV_OK;
     if (!src_key_cache || !src_value_cache || !dst_key_cache || !dst_value_cache || !block_mapping)
@@ -337,10 +339,8 @@ pkv_status pkv_copy_blocks(const void *src_key_cache, const void *src_value_cach
     if (reinterpret_cast<uintptr_t>(block_mapping) & 7u)
         return fail(PKV_ERR_MISALIGNED, "block_mapping must be 8-byte aligned");
     const int64_t vec_per_block = block_bytes / 16;
-    const int64_t n = (int64_t)num_pairs * 2 * vec_per_block;
-    const int threads = 256;
-    const int64_t blocks = std::min<int64_t>((n + threads - 1) / threads, 148 * 16);
-    pkv::copy_blocks_kernel<<<(unsigned)blocks, threads, 0, static_cast<cudaStream_t>(stream)>>>(
+    const int64_t blocks = 2 * (int64_t)num_pairs;   // one CTA per (pair, K or V)
+    pkv::copy_blocks_kernel<<<(unsigned)blocks, pkv::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
         static_cast<const uint4 *>(src_key_cache), static_cast<const uint4 *>(src_value_cache),
         static_cast<uint4 *>(dst_key_cache), static_cast<uint4 *>(dst_value_cache), block_mapping,
         num_pairs, src_num_blocks, dst_num_blocks, vec_per_block);
@@ -696,21 +696,23 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     if (s != PKV_OK)
         return s;
 
-    // merge prefix and suffix records of every (sequence, query head) row
-    constexpr int NT = 512;
+    // merge prefix and suffix records of every (sequence, query head) row:
+    // one warp per row
+    constexpr int NT = 256;
     const int rows = batch * num_heads;
     const int suffix_span = max_suffix_blocks * block_size;
-    auto go = [&](auto kern, int D) {
-        const int ng = NT / D;
-        return launch_pdl(kern, dim3((unsigned)((rows + ng - 1) / ng)), dim3(NT), 0, st, c, a.ws_m,
-                          a.ws_l, a.ws_o, suffix_lens, plan.ps, a.part_tokens, suffix_span, a.out);
+    auto go = [&](auto kern) {
+        constexpr int rows_per_cta = NT / 32;
+        return launch_pdl(kern, dim3((unsigned)((rows + rows_per_cta - 1) / rows_per_cta)), dim3(NT), 0,
+                          st, c, a.ws_m, a.ws_l, a.ws_o, suffix_lens, plan.ps, a.part_tokens,
+                          suffix_span, a.out);
     };
     if (dtype == PKV_BF16)
-        e = head_dim == 64 ? go(pkv::lse_merge_cascade_kernel<true, 64, NT>, 64)
-                           : go(pkv::lse_merge_cascade_kernel<true, 128, NT>, 128);
+        e = head_dim == 64 ? go(pkv::lse_merge_cascade_kernel<true, 64, NT>)
+                           : go(pkv::lse_merge_cascade_kernel<true, 128, NT>);
     else
-        e = head_dim == 64 ? go(pkv::lse_merge_cascade_kernel<false, 64, NT>, 64)
-                           : go(pkv::lse_merge_cascade_kernel<false, 128, NT>, 128);
+        e = head_dim == 64 ? go(pkv::lse_merge_cascade_kernel<false, 64, NT>)
+                           : go(pkv::lse_merge_cascade_kernel<false, 128, NT>);
     if (e != cudaSuccess)
         return cuda_fail(e, "lse_merge_cascade_kernel launch");
     return PKV_OK;

@@ -567,7 +567,22 @@ struct CascadeArgs {
 
 // Cascade merge: row (b, h) = its group's prefix records (partitions of the
 // prefix) and its own suffix records (partitions of the suffix), folded by
-// log-sum-exp.  NT threads = NG groups of D, one row per group.
+// log-sum-exp.  One warp per row, lane = D/32 consecutive columns.  The
+// warp finds the row's group with a 32-way search of group_start (one or two
+// load rounds), spreads the records' (m, l) over its lanes to take the
+// maximum and the weights, then loads every record's O slice independently.
+template <int D>
+__device__ __forceinline__ void load_slice(const float *p, float (&v)[D / 32])
+{
+    if constexpr (D == 128) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(p));
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else {
+        const float2 x = __ldg(reinterpret_cast<const float2 *>(p));
+        v[0] = x.x; v[1] = x.y;
+    }
+}
+
 template <bool BF16, int D, int NT>
 __global__ void __launch_bounds__(NT)
 lse_merge_cascade_kernel(const CascadeArgs c, const float *__restrict__ sm, const float *__restrict__ sl,
@@ -575,23 +590,35 @@ lse_merge_cascade_kernel(const CascadeArgs c, const float *__restrict__ sm, cons
                          int suffix_parts, int suffix_part_tokens, int suffix_span,
                          uint16_t *__restrict__ out)
 {
-    constexpr int NG = NT / D;
+    constexpr int VPT = D / 32;
+    static_assert(D == 64 || D == 128, "head_dim 64 or 128");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int d = threadIdx.x % D;
-    const size_t row = (size_t)blockIdx.x * NG + threadIdx.x / D;
+    const int lane = threadIdx.x & 31;
+    const size_t row = (size_t)blockIdx.x * (NT / 32) + threadIdx.x / 32;
     if (row >= (size_t)c.batch * c.num_heads)
-        return;
+        return;                                  // whole warp
     const int b = (int)(row / c.num_heads);
-    // group of sequence b: the last g with group_start[g] <= b
-    int lo = 0, hi = c.num_groups - 1, g = -1;
-    while (lo <= hi) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(c.group_start + mid) <= b) {
-            g = mid;
-            lo = mid + 1;
-        } else {
-            hi = mid - 1;
+
+    // group of sequence b: the last g with group_start[g] <= b (starts ascend)
+    int lo = 0, n = c.num_groups;                // candidates lo .. lo + n - 1
+    while (n > 32) {
+        const int step = (n + 31) / 32;
+        const int idx = lo + lane * step;
+        const unsigned le = __ballot_sync(0xffffffffu, idx < lo + n && __ldg(c.group_start + idx) <= b);
+        if (le == 0u) {
+            n = 0;                               // every candidate starts after b
+            break;
         }
+        const int nlo = lo + (31 - __clz(le)) * step;
+        n = min(step, lo + n - nlo);
+        lo = nlo;
+    }
+    int g = lo - 1;
+    if (n > 0) {
+        const unsigned le =
+            __ballot_sync(0xffffffffu, lane < n && __ldg(c.group_start + lo + lane) <= b);
+        if (le != 0u)
+            g = lo + 31 - __clz(le);
     }
     int np_p = 0;
     if (g >= 0 && b < __ldg(c.group_start + g + 1)) {
@@ -602,29 +629,64 @@ lse_merge_cascade_kernel(const CascadeArgs c, const float *__restrict__ sm, cons
     int Ls = __ldg(suffix_lens + b);
     Ls = Ls < 0 ? 0 : (Ls > suffix_span ? suffix_span : Ls);
     const int np_s = (Ls + suffix_part_tokens - 1) / suffix_part_tokens;
-    float M = kNegInf, den = 0.f, num = 0.f;
-    auto fold = [&](float mp, float lp, float op) {
-        if (!(lp > 0.f))
-            return;
-        if (mp > M) {
-            const float sc = ex2(M - mp);
-            den *= sc;
-            num *= sc;
-            M = mp;
-        }
-        const float w = ex2(mp - M) * lp;
-        den += w;
-        num += w * op;
+    const int nrec = np_p + np_s;               // record k: prefix k, then suffix k - np_p
+
+    // record k's (m, l) and O slice
+    auto rec_ml = [&](int k, float &m, float &l) {
+        const size_t r = k < np_p ? row * c.num_parts + k : row * suffix_parts + (k - np_p);
+        m = __ldg((k < np_p ? c.rec_m : sm) + r);
+        l = __ldg((k < np_p ? c.rec_l : sl) + r);
     };
-    for (int p = 0; p < np_p; ++p) {
-        const size_t rec = row * c.num_parts + p;
-        fold(__ldg(c.rec_m + rec), __ldg(c.rec_l + rec), __ldg(c.rec_o + rec * D + d));
+    auto rec_o = [&](int k) {
+        return k < np_p ? c.rec_o + (row * c.num_parts + k) * D : so + (row * suffix_parts + (k - np_p)) * D;
+    };
+
+    // the maximum over records that hold keys (l > 0)
+    float M = kNegInf;
+    for (int k0 = 0; k0 < nrec; k0 += 32) {
+        float m = kNegInf, l = 0.f;
+        if (k0 + lane < nrec)
+            rec_ml(k0 + lane, m, l);
+        if (l > 0.f)
+            M = fmaxf(M, m);
     }
-    for (int p = 0; p < np_s; ++p) {
-        const size_t rec = row * suffix_parts + p;
-        fold(__ldg(sm + rec), __ldg(sl + rec), __ldg(so + rec * D + d));
+#pragma unroll
+    for (int off = 16; off; off >>= 1)
+        M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    // weights w_k = 2^(m_k - M) l_k, spread over the lanes; den = sum w_k
+    float den = 0.f, acc[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+        acc[i] = 0.f;
+    for (int k0 = 0; k0 < nrec; k0 += 32) {
+        float m = kNegInf, l = 0.f;
+        if (k0 + lane < nrec)
+            rec_ml(k0 + lane, m, l);
+        const float w = l > 0.f ? ex2(m - M) * l : 0.f;
+        den += w;
+        const int nk = min(32, nrec - k0);
+        for (int k = 0; k < nk; ++k) {
+            const float wk = __shfl_sync(0xffffffffu, w, k);
+            if (wk > 0.f) {                      // warp-uniform
+                float v[VPT];
+                load_slice<D>(rec_o(k0 + k) + lane * VPT, v);
+#pragma unroll
+                for (int i = 0; i < VPT; ++i)
+                    acc[i] += wk * v[i];
+            }
+        }
     }
-    out[row * D + d] = to_storage<BF16>(den > 0.f ? num / den : 0.f);
+#pragma unroll
+    for (int off = 16; off; off >>= 1)
+        den += __shfl_xor_sync(0xffffffffu, den, off);
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    uint16_t *o = out + row * D + lane * VPT;
+    if constexpr (VPT == 4) {
+        *reinterpret_cast<uint2 *>(o) = make_uint2(pack2<BF16>(acc[0] * inv, acc[1] * inv),
+                                                   pack2<BF16>(acc[2] * inv, acc[3] * inv));
+    } else {
+        *reinterpret_cast<uint32_t *>(o) = pack2<BF16>(acc[0] * inv, acc[1] * inv);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -638,30 +700,43 @@ lse_merge_cascade_kernel(const CascadeArgs c, const float *__restrict__ sm, cons
 // V, as 16-byte vectors; either side may be pinned host memory (reached
 // through unified addressing).  Pairs naming a block outside its pool are
 // skipped and set PKV_DEVFLAG_BLOCK_RANGE.
-__global__ void copy_blocks_kernel(const uint4 *__restrict__ src_k, const uint4 *__restrict__ src_v,
-                                   uint4 *__restrict__ dst_k, uint4 *__restrict__ dst_v,
-                                   const int32_t *__restrict__ mapping, int num_pairs,
-                                   int64_t src_blocks, int64_t dst_blocks, int64_t vec_per_block)
+// One CTA per (pair, K or V): 256 threads move the block's 16-byte vectors,
+// kCopyUnroll loads in flight per thread before their stores.
+constexpr int kCopyThreads = 256;
+constexpr int kCopyUnroll = 8;
+__global__ void __launch_bounds__(kCopyThreads)
+copy_blocks_kernel(const uint4 *__restrict__ src_k, const uint4 *__restrict__ src_v,
+                   uint4 *__restrict__ dst_k, uint4 *__restrict__ dst_v,
+                   const int32_t *__restrict__ mapping, int num_pairs, int64_t src_blocks,
+                   int64_t dst_blocks, int64_t vec_per_block)
 {
-    const int64_t per_pair = 2 * vec_per_block;   // K then V
-    const int64_t n = (int64_t)num_pairs * per_pair;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-        const int64_t pair = i / per_pair;
-        int64_t v = i - pair * per_pair;
-        const bool is_v = v >= vec_per_block;
-        v -= is_v ? vec_per_block : 0;
-        const int64_t s = __ldg(mapping + 2 * pair);
-        const int64_t d = __ldg(mapping + 2 * pair + 1);
-        if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) {
-            if (v == 0 && !is_v)
-                raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
-            continue;
+    const int64_t pair = blockIdx.x >> 1;
+    const bool is_v = blockIdx.x & 1;
+    if (pair >= num_pairs)
+        return;
+    const int64_t s = __ldg(mapping + 2 * pair);
+    const int64_t d = __ldg(mapping + 2 * pair + 1);
+    if (s < 0 || s >= src_blocks || d < 0 || d >= dst_blocks) {
+        if (threadIdx.x == 0 && !is_v)
+            raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
+        return;                                  // the pair is skipped
+    }
+    const uint4 *src = (is_v ? src_v : src_k) + s * vec_per_block;
+    uint4 *dst = (is_v ? dst_v : dst_k) + d * vec_per_block;
+    for (int64_t v0 = threadIdx.x; v0 < vec_per_block; v0 += kCopyThreads * kCopyUnroll) {
+        uint4 r[kCopyUnroll];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t v = v0 + u * kCopyThreads;
+            if (v < vec_per_block)
+                r[u] = src[v];
         }
-        if (is_v)
-            dst_v[d * vec_per_block + v] = src_v[s * vec_per_block + v];
-        else
-            dst_k[d * vec_per_block + v] = src_k[s * vec_per_block + v];
+#pragma unroll
+        for (int u = 0; u < kCopyUnroll; ++u) {
+            const int64_t v = v0 + u * kCopyThreads;
+            if (v < vec_per_block)
+                dst[v] = r[u];
+        }
     }
 }
 
