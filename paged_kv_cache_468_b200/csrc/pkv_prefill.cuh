@@ -285,18 +285,20 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                     ids = kb0 + lane < nblk ? __ldg(trow + kb0 + lane) : 0;
                 if (lane == 0)
                     mbar_arrive_expect_tx(bar(full0 + s), (uint32_t)(nb * BS * D * 2));
-                for (int i = 0; i < nb; ++i) {
-                    int blk = __shfl_sync(0xffffffffu, ids, (kb0 + i) & 31);
-                    if (lane == 0) {
-                        if ((unsigned)blk >= (unsigned)num_blocks) {
+                __syncwarp();
+                // lane i * kHalves + h copies half h of the tile's block i: the
+                // tile's copies leave in one warp instruction, not one by one
+                const int i = lane / Sh::kHalves;
+                const int h = lane - i * Sh::kHalves;
+                int blk = __shfl_sync(0xffffffffu, ids, (kb0 + min(i, BPT - 1)) & 31);
+                if (i < nb) {
+                    if ((unsigned)blk >= (unsigned)num_blocks) {
+                        if (h == 0)
                             raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
-                            blk = 0;
-                        }
-#pragma unroll
-                        for (int h = 0; h < Sh::kHalves; ++h)
-                            tma_load_3d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
-                                        bar(full0 + s), h * 64, kvh, blk * BS, policy);
+                        blk = 0;
                     }
+                    tma_load_3d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
+                                bar(full0 + s), h * 64, kvh, blk * BS, policy);
                 }
                 issued = j + 1;
             }
