@@ -39,6 +39,7 @@ from paged_kv_cache_468_b200 import workloads  # noqa: E402
 
 METRIC = "paged decode attention KV GB/s (fraction of B200 HBM peak); decode tokens/s"
 KERNEL_SOURCES = ["paged_kv_cache_468_b200/csrc/pkv_kernels.cuh",
+                  "paged_kv_cache_468_b200/csrc/pkv_prefill.cuh",
                   "paged_kv_cache_468_b200/csrc/pkv_ptx.cuh",
                   "paged_kv_cache_468_b200/csrc/pagedkv.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
