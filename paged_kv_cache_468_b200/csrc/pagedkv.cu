@@ -165,10 +165,10 @@ cudaError_t launch_merge_d(const pkv::DecodeArgs &a, const int32_t *context_lens
 {
     constexpr int NT = 512, NG = NT / D;
     if (np <= 8)
-        return launch_pdl(pkv::lse_merge_kernel<BF16, D, NT, NG>, dim3((unsigned)((rows + NG - 1) / NG)),
+        return launch_pdl(pkv::lse_merge_kernel<BF16, D, NT>, dim3((unsigned)((rows + NG - 1) / NG)),
                           dim3(NT), 0, st, a.ws_m, a.ws_l, a.ws_o, context_lens, Hq, rows, np, pt,
                           span, a.out);
-    return launch_pdl(pkv::lse_merge_kernel<BF16, D, NT, 1>, dim3((unsigned)rows), dim3(NT), 0, st,
+    return launch_pdl(pkv::lse_merge_wide_kernel<BF16, D, NT>, dim3((unsigned)rows), dim3(NT), 0, st,
                       a.ws_m, a.ws_l, a.ws_o, context_lens, Hq, rows, np, pt, span, a.out);
 }
 

@@ -87,6 +87,19 @@ __device__ __forceinline__ uint16_t to_storage(float x)
     }
 }
 
+// D/32 consecutive floats of a record, one lane's share
+template <int D>
+__device__ __forceinline__ void load_slice(const float *p, float (&v)[D / 32])
+{
+    if constexpr (D == 128) {
+        const float4 x = __ldg(reinterpret_cast<const float4 *>(p));
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else {
+        const float2 x = __ldg(reinterpret_cast<const float2 *>(p));
+        v[0] = x.x; v[1] = x.y;
+    }
+}
+
 // ---------------------------------------------------------------------------
 // KV write through slot_mapping ([MH] 2.1, 3.3)
 // ---------------------------------------------------------------------------
@@ -571,18 +584,6 @@ struct CascadeArgs {
 // warp finds the row's group with a 32-way search of group_start (one or two
 // load rounds), spreads the records' (m, l) over its lanes to take the
 // maximum and the weights, then loads every record's O slice independently.
-template <int D>
-__device__ __forceinline__ void load_slice(const float *p, float (&v)[D / 32])
-{
-    if constexpr (D == 128) {
-        const float4 x = __ldg(reinterpret_cast<const float4 *>(p));
-        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
-    } else {
-        const float2 x = __ldg(reinterpret_cast<const float2 *>(p));
-        v[0] = x.x; v[1] = x.y;
-    }
-}
-
 template <bool BF16, int D, int NT>
 __global__ void __launch_bounds__(NT)
 lse_merge_cascade_kernel(const CascadeArgs c, const float *__restrict__ sm, const float *__restrict__ sl,
@@ -761,30 +762,28 @@ __global__ void bounded_wait_selftest_kernel(uint64_t limit_ns)
 // ---------------------------------------------------------------------------
 // Log-sum-exp merge of split partitions
 // ---------------------------------------------------------------------------
-// One CTA per RPC (sequence, query head) rows.  NT threads = NG groups of D.  With RPC == NG each group merges its own
-// (sequence, query head) row over all of its partitions (plans with few
-// partitions: fewer, fuller CTAs); with RPC == 1 the groups fold one row's
-// partitions q, q + NG, ... with an online log-sum-exp and are then combined
-// (plans with many partitions).  out = sum_p w_p o_p / sum_p w_p,
-// w_p = 2^(m_p - M) l_p, M = max_p m_p, over the partitions that hold tokens.
-// Launched with programmatic dependent launch: it waits for the decode first.
-template <bool BF16, int D, int NT, int RPC>
+// out = sum_p w_p o_p / sum_p w_p, w_p = 2^(m_p - M) l_p, M = max_p m_p, over
+// the partitions of a (sequence, query head) row that hold tokens, with an
+// online log-sum-exp.  Two launch shapes: lse_merge_kernel for plans with few
+// partitions (several rows per CTA, a thread per column), lse_merge_wide_kernel
+// for many (a CTA per row, its warps folding interleaved partitions, then
+// combined).  Launched with programmatic dependent launch: they wait for the
+// decode first.
+
+template <bool BF16, int D, int NT>
 __global__ void __launch_bounds__(NT)
 lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
                  const float *__restrict__ ws_o, const int32_t *__restrict__ context_lens,
                  int num_heads, int num_rows, int num_parts, int part_tokens, int span,
                  uint16_t *__restrict__ out)
 {
+    // few partitions: NT / D rows per CTA, thread = one column of one row
     constexpr int NG = NT / D;
-    static_assert(RPC == 1 || RPC == NG, "rows per CTA");
-    __shared__ float s_M[NG][D], s_den[NG][D], s_num[NG][D];
     asm volatile("griddepcontrol.wait;" ::: "memory");
-
     const int d = threadIdx.x % D;
-    const int grp = threadIdx.x / D;
-    const size_t row = (size_t)blockIdx.x * RPC + (RPC == 1 ? 0 : grp);
+    const size_t row = (size_t)blockIdx.x * NG + threadIdx.x / D;
     if (row >= (size_t)num_rows)
-        return;                                  // (RPC > 1: no barrier follows)
+        return;
     const int b = (int)(row / num_heads);
     int L = __ldg(context_lens + b);
     L = L < 0 ? 0 : (L > span ? span : L);
@@ -792,11 +791,9 @@ lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
     const float *m = ws_m + row * num_parts;
     const float *l = ws_l + row * num_parts;
     const float *o = ws_o + row * num_parts * D + d;
-    const int p0 = RPC == 1 ? grp : 0;
-    const int pstep = RPC == 1 ? NG : 1;
     float M = kNegInf, den = 0.f, num = 0.f;
 #pragma unroll 4
-    for (int p = p0; p < np; p += pstep) {
+    for (int p = 0; p < np; ++p) {
         const float mp = __ldg(m + p);
         const float lp = __ldg(l + p);
         const float op = __ldg(o + (size_t)p * D);
@@ -810,27 +807,98 @@ lse_merge_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
         den += w;
         num += w * op;
     }
-    if (RPC > 1) {
-        out[row * D + d] = to_storage<BF16>(den > 0.f ? num / den : 0.f);
-        return;
+    out[row * D + d] = to_storage<BF16>(den > 0.f ? num / den : 0.f);
+}
+
+// Many partitions: one CTA per row; NG groups of 32 threads, group g folds the
+// partitions p = g, g + NG, ... (a thread holds D/32 consecutive columns, so a
+// group's loads of one partition are independent of its other partitions'),
+// then group 0 folds the NG partial results.
+template <bool BF16, int D, int NT>
+__global__ void __launch_bounds__(NT)
+lse_merge_wide_kernel(const float *__restrict__ ws_m, const float *__restrict__ ws_l,
+                      const float *__restrict__ ws_o, const int32_t *__restrict__ context_lens,
+                      int num_heads, int num_rows, int num_parts, int part_tokens, int span,
+                      uint16_t *__restrict__ out)
+{
+    constexpr int VPT = D / 32;
+    constexpr int NG = NT / 32;
+    __shared__ float s_M[NG], s_den[NG];
+    __shared__ __align__(16) float s_num[NG][D];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const int lane = threadIdx.x & 31;
+    const int grp = threadIdx.x >> 5;
+    const size_t row = blockIdx.x;
+    if (row >= (size_t)num_rows)
+        return;                                  // whole CTA
+    const int b = (int)(row / num_heads);
+    int L = __ldg(context_lens + b);
+    L = L < 0 ? 0 : (L > span ? span : L);
+    const int np = (L + part_tokens - 1) / part_tokens;
+    const float *m = ws_m + row * num_parts;
+    const float *l = ws_l + row * num_parts;
+    const float *o = ws_o + row * num_parts * D + lane * VPT;
+    float M = kNegInf, den = 0.f, num[VPT];
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+        num[i] = 0.f;
+#pragma unroll 4
+    for (int p = grp; p < np; p += NG) {
+        const float mp = __ldg(m + p);
+        const float lp = __ldg(l + p);
+        float v[VPT];
+        load_slice<D>(o + (size_t)p * D, v);
+        if (mp > M) {
+            const float sc = ex2(M - mp);       // 0 while M is -inf
+            den *= sc;
+#pragma unroll
+            for (int i = 0; i < VPT; ++i)
+                num[i] *= sc;
+            M = mp;
+        }
+        const float w = ex2(mp - M) * lp;
+        den += w;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+            num[i] += w * v[i];
     }
-    s_M[grp][d] = M;
-    s_den[grp][d] = den;
-    s_num[grp][d] = num;
+    if (lane == 0) {
+        s_M[grp] = M;
+        s_den[grp] = den;
+    }
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+        s_num[grp][lane * VPT + i] = num[i];
     __syncthreads();
     if (grp == 0) {
         float Mt = kNegInf;
 #pragma unroll
         for (int q = 0; q < NG; ++q)
-            Mt = fmaxf(Mt, s_M[q][d]);
-        float dt = 0.f, nt = 0.f;
+            Mt = fmaxf(Mt, s_M[q]);
+        float dt = 0.f, nt[VPT];
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+            nt[i] = 0.f;
 #pragma unroll
         for (int q = 0; q < NG; ++q) {
-            const float e = ex2(s_M[q][d] - Mt);   // 0 for groups that held no partition
-            dt += e * s_den[q][d];
-            nt += e * s_num[q][d];
+            // 0 for groups that held no partition (also when none did: no NaN)
+            const float e = s_M[q] == kNegInf ? 0.f : ex2(s_M[q] - Mt);
+            dt += e * s_den[q];
+#pragma unroll
+            for (int i = 0; i < VPT; ++i)
+                nt[i] += e * s_num[q][lane * VPT + i];
         }
-        out[row * D + d] = to_storage<BF16>(dt > 0.f ? nt / dt : 0.f);
+        const float inv = dt > 0.f ? 1.f / dt : 0.f;
+#pragma unroll
+        for (int i = 0; i < VPT; ++i)
+            nt[i] = dt > 0.f ? nt[i] * inv : 0.f;
+        uint16_t *op = out + row * D + lane * VPT;
+        if constexpr (VPT == 4) {
+            *reinterpret_cast<uint2 *>(op) =
+                make_uint2(pack2<BF16>(nt[0], nt[1]), pack2<BF16>(nt[2], nt[3]));
+        } else {
+            *reinterpret_cast<uint32_t *>(op) = pack2<BF16>(nt[0], nt[1]);
+        }
     }
 }
 

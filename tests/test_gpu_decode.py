@@ -132,6 +132,16 @@ def test_empty_context_gives_zeros():
     assert torch.count_nonzero(out[0]) == 0
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_empty_context_many_partitions(D):
+    """13 partitions per row (the merge that gives each row a CTA): rows
+    without tokens still come out as zeros, next to a row that has them."""
+    step = custom("empty_wide", 3, 8, 8, D, 16, "bf16", [0, 200, 0], seed=13)
+    step["slot_mapping"][:] = -1
+    out, _ = _parity(step, write=False, partition_tokens=16)
+    assert torch.count_nonzero(out[0]) == 0 and torch.count_nonzero(out[2]) == 0
+
+
 def test_shared_prefix_tables_from_allocator():
     """Forked samples share the prefix blocks (refcounted, read-only); the
     decode equals the oracle on the allocator's tables."""
