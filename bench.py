@@ -38,10 +38,6 @@ sys.path.insert(0, ROOT)
 from paged_kv_cache_468_b200 import workloads  # noqa: E402
 
 METRIC = "paged decode attention KV GB/s (fraction of B200 HBM peak); decode tokens/s"
-KERNEL_SOURCES = ["paged_kv_cache_468_b200/csrc/pkv_kernels.cuh",
-                  "paged_kv_cache_468_b200/csrc/pkv_prefill.cuh",
-                  "paged_kv_cache_468_b200/csrc/pkv_ptx.cuh",
-                  "paged_kv_cache_468_b200/csrc/pagedkv.cu"]
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
 FALLBACK_HBM_GBS = 6650.0
 
@@ -89,24 +85,89 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": FALLBACK_HBM_GBS, "source": "fallback"}
 
 
-def kernel_source_sha() -> str:
+# The DRAM traffic recorded for a workload's decode call (ncu) stays valid
+# while the source text of the code that call runs is unchanged: the PTX
+# wrappers, and the named functions / structs below.
+CSRC = "paged_kv_cache_468_b200/csrc/"
+_DECODE_CODE = [
+    ("pkv_kernels.cuh", ["DecodeArgs", "DecodeShape", "pack2", "unpack2", "to_storage",
+                         "attend_block", "paged_decode_kernel"]),
+    ("pagedkv.cu", ["Tuning", "make_cache_map", "check_shapes", "plan", "launch_pdl",
+                    "launch_decode", "dispatch_decode", "pkv_paged_attention_decode"]),
+]
+_SPLIT_CODE = [
+    ("pkv_kernels.cuh", ["load_slice", "lse_merge_kernel", "lse_merge_wide_kernel"]),
+    ("pagedkv.cu", ["launch_merge_d", "launch_merge"]),
+]
+_CASCADE_CODE = [
+    ("pkv_kernels.cuh", ["CascadeArgs", "load_slice", "lse_merge_cascade_kernel"]),
+    ("pkv_prefill.cuh", ["PrefillArgs", "PfShape", "PfBar", "tc_attend", "prefix_tc_kernel"]),
+    ("pagedkv.cu", ["make_query_map", "cascade_plan", "launch_prefix", "dispatch_prefix",
+                    "pkv_paged_attention_decode_cascade"]),
+]
+
+
+def _definitions(src: str, name: str) -> list:
+    """Source text of every definition of function / struct / enum `name`
+    (with the template and attribute lines above it)."""
+    import re
+    out = []
+    for m in re.finditer(r"\b(?:struct|enum)\s+" + re.escape(name) + r"\b[^;{]*\{|\b" + re.escape(name) + r"\s*\(", src):
+        i = m.end()
+        if src[m.end() - 1] == "(":                       # function: its parameter list
+            depth = 1
+            while i < len(src) and depth:
+                depth += {"(": 1, ")": -1}.get(src[i], 0)
+                i += 1
+            j = i
+            while j < len(src) and (src[j].isspace() or src[j:j + 5] in ("const", "noexc")):
+                j += 5 if src[j:j + 5] in ("const", "noexc") else 1
+            if j >= len(src) or src[j] != "{":
+                continue                                  # a call or a declaration
+            i = j + 1
+        depth = 1
+        while i < len(src) and depth:
+            depth += {"{": 1, "}": -1}.get(src[i], 0)
+            i += 1
+        start = src.rfind("\n", 0, m.start()) + 1
+        while start > 0:                                  # template / attribute lines above
+            prev = src.rfind("\n", 0, start - 1) + 1
+            line = src[prev:start - 1].strip()
+            if not line or line.endswith((";", "}", "{")) or line.startswith("//"):
+                break
+            start = prev
+        out.append(src[start:i])
+    if not out:
+        raise KeyError(name)
+    return out
+
+
+def decode_code_sha(split: bool, cascade: bool, root: str = ROOT) -> str:
+    """Fingerprint of the code a decode call runs (16 hex digits)."""
+    parts = list(_DECODE_CODE) + (list(_SPLIT_CODE) if split else []) + \
+        (list(_CASCADE_CODE) if cascade else [])
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+    with open(os.path.join(root, CSRC, "pkv_ptx.cuh"), "rb") as f:
+        h.update(f.read())
+    for fname, names in parts:
+        with open(os.path.join(root, CSRC, fname), encoding="utf-8") as f:
+            src = f.read()
+        for n in names:
+            for text in _definitions(src, n):
+                h.update(text.encode())
     return h.hexdigest()[:16]
 
 
-def committed_traffic(config_name: str):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel sources and this workload (else None)."""
+def committed_traffic(config_name: str, split: bool, cascade: bool):
+    """DRAM bytes per decode call from the committed ncu summary, if they were
+    taken on the code this call runs now (else None)."""
     try:
         with open(TRAFFIC_FILE) as f:
             d = json.load(f)
     except (OSError, ValueError):
         return None
     entry = d.get(config_name)
-    if not entry or entry.get("source_sha") != kernel_source_sha():
+    if not entry or entry.get("source_sha") != decode_code_sha(split, cascade):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -480,7 +541,7 @@ def run_gpu(args, cfg, world, rank, local):
     achieved = nbytes["decode_unique"] / (decode_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": committed_traffic(cfg.name),
+                "traffic": committed_traffic(cfg.name, plan_np > 1 and not cascade, cascade),
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
                 if peaks["source"] == "measured" else "fallback 6650 GB/s",
                 "kernel": ("prefix_tc_kernel + paged_decode_kernel (suffixes) + "
