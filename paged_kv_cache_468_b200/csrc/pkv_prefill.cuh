@@ -10,8 +10,10 @@
 // section 三); query token i sits at position L_b - C_b + i and attends
 // causally over tokens 0 .. L_b - C_b + i of its paged cache.
 //
-// One CTA per (row tile, kv head, sequence).  A row is a (query token, head
-// of the kv head's GQA group) pair, 128 rows per CTA (the M of every MMA).
+// One CTA per (row tile, kv head, sequence); for the prefix pass, per
+// (prefix partition, kv head, chunk of 128/G group members).  A row is a
+// (query token or group member, head of the kv head's GQA group) pair, 128
+// rows per CTA (the M of every MMA).
 // Keys are taken 64 at a time (a "key tile": 64 / block_size cache blocks
 // located through the block table, exactly as the decode kernels do):
 //
@@ -25,7 +27,8 @@
 // by more than 2^8 (P then stays <= 256); O and the row sum are rescaled by
 // the softmax warps at that point, so the result equals the one-pass softmax
 // up to rounding.  S (and P over it) is double-buffered in TMEM: the
-// softmax of tile j+1 reads its scores while P_j V_j runs.
+// softmax of tile j+1 reads its scores while P_j V_j runs, and stores P_{j+1}
+// once P_j V_j has completed (no MMA runs while TMEM is written).
 // Warp roles: 0-3 softmax + epilogue (warp w owns TMEM lanes 32w..32w+31),
 // 4 loads Q and the K ring (3 stages), 5 allocates TMEM and issues every MMA,
 // 6 loads the V ring (2 stages) and clears V rows past the last visible key
