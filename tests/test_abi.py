@@ -137,3 +137,41 @@ def test_cascade_workspace_and_validation():
     assert L.pkv_paged_attention_decode_cascade(None, None, None, None, 4, None, None, 1, 2, None, 4,
                                                 None, 2, 8, 8, 64, 16, 100, 1.0, 0, None, 0, None,
                                                 1, None) == pagedkv.ERR_INVALID_ARG
+
+
+def test_prefill_host_validation():
+    L = pkv.lib()
+    a16 = 0x10000
+    # query, num_tokens, query_start, max_query_len, key_cache, value_cache, block_tables,
+    # max_blocks, context_lens, batch, Hq, Hkv, D, bs, num_blocks, scale, out, dtype, stream
+    def call(q=a16, T=64, qs=a16, mql=32, kc=a16, vc=a16, bt=a16, mb=8, cl=a16, B=2, Hq=8, Hkv=2,
+             D=128, bs=16, nb=100, scale=0.125, out=a16, dt=1):
+        return L.pkv_paged_attention_prefill(q, T, qs, mql, kc, vc, bt, mb, cl, B, Hq, Hkv, D, bs, nb,
+                                             scale, out, dt, None)
+    assert call(Hq=32, Hkv=2) == pagedkv.ERR_UNSUPPORTED           # group 16 > 8
+    assert call(D=96) == pagedkv.ERR_UNSUPPORTED
+    assert call(dt=7) == pagedkv.ERR_INVALID_ARG
+    assert call(T=-1) == pagedkv.ERR_INVALID_ARG
+    assert call(mql=8 * 16 + 1) == pagedkv.ERR_INVALID_ARG         # > max_blocks * block_size
+    assert call(nb=0) == pagedkv.ERR_INVALID_ARG
+    assert call(scale=float("inf")) == pagedkv.ERR_INVALID_ARG
+    assert call(q=None, qs=None, kc=None, vc=None, bt=None, cl=None, out=None, B=0) == pagedkv.OK
+    assert call(T=0, q=None, out=None) == pagedkv.OK                # nothing to do
+    assert call(out=None) == pagedkv.ERR_INVALID_ARG
+    assert call(q=a16 + 8) == pagedkv.ERR_MISALIGNED
+
+
+def test_copy_blocks_host_validation():
+    L = pkv.lib()
+    a16 = 0x10000
+    # src_k, src_v, dst_k, dst_v, mapping, num_pairs, src_blocks, dst_blocks, block_bytes, stream
+    def call(p=a16, m=a16, n=4, sb=10, db=10, bb=16 * 8 * 128 * 2):
+        return L.pkv_copy_blocks(p, p, p, p, m, n, sb, db, bb, None)
+    assert call(n=-1) == pagedkv.ERR_INVALID_ARG
+    assert call(sb=0) == pagedkv.ERR_INVALID_ARG
+    assert call(bb=24) == pagedkv.ERR_UNSUPPORTED                   # not a multiple of 16
+    assert call(n=(1 << 30) + 1) == pagedkv.ERR_UNSUPPORTED         # grid of 2 CTAs per pair
+    assert call(n=0, p=None, m=None) == pagedkv.OK
+    assert call(m=None) == pagedkv.ERR_INVALID_ARG
+    assert call(p=a16 + 8) == pagedkv.ERR_MISALIGNED
+    assert call(m=a16 + 4) == pagedkv.ERR_MISALIGNED
