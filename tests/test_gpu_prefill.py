@@ -73,8 +73,9 @@ def test_prefill_last_token_equals_decode():
     assert (out[qs[1:].long().cuda() - 1].float() - dec.float()).abs().max().item() <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("dtype", ["f16", "bf16"])
-def test_prefill_growing_scores(dtype):
+def test_prefill_growing_scores(dtype, D):
     """Keys grow along the context, so each row's running maximum keeps
     moving by more than 2^8 in weight: every rescale of the running output
     is exercised, and the result must still be the one-pass softmax.  The
@@ -82,7 +83,7 @@ def test_prefill_growing_scores(dtype):
     entries; V is scaled by 1/4 to keep them below 2, where rounding the
     output to the storage type stays inside the fixed absolute bound."""
     lens, chunks = [900, 333], [600, 333]
-    step, q, qs = _case(lens, chunks, 8, 2, 128, 16, dtype, seed=5)
+    step, q, qs = _case(lens, chunks, 8, 2, D, 16, dtype, seed=5)
     kc = step["key_cache"].float()
     tables = step["block_tables"]
     for s_, L in enumerate(lens):
