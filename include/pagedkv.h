@@ -132,8 +132,11 @@ pkv_status pkv_kv_cache_write(const void *key, const void *value,
  * memory or pinned host memory (reached through unified addressing), so the
  * same call does copy-on-write inside one pool (source = destination caches),
  * swap-out to host and swap-in.  block_bytes = block_size * num_kv_heads *
- * head_dim * 2, a multiple of 16.  Destination blocks must be distinct and
- * not also sources in the same call.  Out-of-range pairs are skipped and set
+ * head_dim * 2, a multiple of 16 (else PKV_ERR_UNSUPPORTED).  Destination
+ * blocks must be distinct and not also sources in the same call.  num_pairs
+ * is at most 2^30 (one CTA per pair and K or V; else PKV_ERR_UNSUPPORTED);
+ * caches 16-byte aligned and the mapping 8-byte aligned (else
+ * PKV_ERR_MISALIGNED).  Out-of-range pairs are skipped and set
  * PKV_DEVFLAG_BLOCK_RANGE.
  */
 pkv_status pkv_copy_blocks(const void *src_key_cache, const void *src_value_cache,
