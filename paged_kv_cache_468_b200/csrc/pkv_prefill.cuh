@@ -27,8 +27,22 @@
 // by more than 2^8 (P then stays <= 256); O and the row sum are rescaled by
 // the softmax warps at that point, so the result equals the one-pass softmax
 // up to rounding.  S (and P over it) is double-buffered in TMEM: the
-// softmax of tile j+1 reads its scores while P_j V_j runs, and stores P_{j+1}
-// once P_j V_j has completed (no MMA runs while TMEM is written).
+// tensor core computes S_{j+1} while the softmax warps work on tile j.
+//
+// Ordering (tcgen05 keeps back-to-back MMAs in issue order only when they
+// share the accumulator and the shape; S and O differ in both):
+//   * S_{j+1} overwrites the buffer that holds P_{j-1}, the A operand of
+//     P_{j-1} V_{j-1}: the MMA thread issues S_{j+1} only after that MMA has
+//     completed (O_DONE of tile j-1).
+//   * The softmax warps store P_j only after P_{j-1} V_{j-1} has completed:
+//     O is then stable for a rescale, and O_DONE (one barrier, one phase per
+//     tile) is never more than one phase ahead of any wait on it.  Without
+//     this wait the softmax could finish its last tile while two P V phases
+//     were still open, and the epilogue's parity wait for the last phase then
+//     matched the phase two back and read O early (wrong rows in 10-40% of
+//     runs of a 7-token chunk over 520 keys).
+//   * While P_j is stored, the only MMA that can be running is S_{j+1}, which
+//     writes the other buffer.
 // Warp roles: 0-3 softmax + epilogue (warp w owns TMEM lanes 32w..32w+31),
 // 4 loads Q and the K ring (3 stages), 5 allocates TMEM and issues every MMA,
 // 6 loads the V ring (2 stages) and clears V rows past the last visible key
@@ -99,8 +113,8 @@ enum PfBar {
     kNumPfBars = 20
 };
 // A barrier per S/P buffer completes once per two tiles, and buffer j & 1 is
-// refilled (S_{j+2}) only after the MMA thread consumed P_j: no barrier can
-// run two phases ahead of its waiter.
+// refilled (S_{j+2}) only after P_j V_j has completed: no barrier can run two
+// phases ahead of its waiter.
 
 // The body shared by the chunked prefill (PREFIX = false: causal rows of one
 // sequence's chunk) and the prefix pass of cascade decode (PREFIX = true: the
@@ -346,8 +360,9 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             constexpr uint32_t idS = f16_idesc<BF16>(kPfRows, kPfKeys, false);
             constexpr uint32_t idO = f16_idesc<BF16>(kPfRows, D, true);
             // S_j = Q K_j^T into S buffer j & 1; Q and K K-major, 128-byte rows.
-            // Buffer j & 1 last held P_{j-2}, read by P_{j-2} V_{j-2}, issued
-            // earlier by this thread: its MMAs execute in issue order.
+            // Buffer j & 1 last held P_{j-2}, read by P_{j-2} V_{j-2}: an MMA
+            // with another accumulator and shape is not ordered behind it, so
+            // the caller waits for it to complete first.
             auto issue_s = [&](int j) -> bool {
                 const int ks_ = j % kPfKStages;
                 if (!mbar_wait_bounded(bar(kBarKFull + ks_), (uint32_t)((j / kPfKStages) & 1),
@@ -369,8 +384,15 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             };
             bool ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
             for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt && !(ok = issue_s(j + 1)))
-                    break;
+                if (j + 1 < nt) {
+                    // P_{j-1} V_{j-1} reads buffer (j+1) & 1.  O_DONE is at most
+                    // one phase past j-1 here: P_j V_j is not issued yet.
+                    if (j >= 1 &&
+                        !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs)))
+                        break;
+                    if (!(ok = issue_s(j + 1)))
+                        break;
+                }
                 const int vs = j % kPfVStages;
                 ok = mbar_wait_bounded(bar(kBarPFull + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
                      mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((j / kPfVStages) & 1),
@@ -467,13 +489,12 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             l = l * alpha + rs;
             m_used = m_new;
             if (j > 0) {
-                // P_j is stored only once P_{j-1} V_{j-1} has completed, so no
-                // MMA is running when TMEM is written (and O holds P_{j-1} V_{j-1}
-                // for a rescale).  Storing P_j while that MMA was still running
-                // gave intermittently wrong rows on B200 (10-40% of runs of a
-                // 7-token chunk over 520 keys); with the wait, none in hundreds
-                // of runs.  O_DONE is at most one phase ahead of this wait:
-                // P_j V_j needs this warp's P_j.
+                // Wait for P_{j-1} V_{j-1}: O then holds it (for the rescale),
+                // and O_DONE stays within one phase of this warp, so the
+                // epilogue's parity wait below names the last tile's phase and
+                // no other.  O_DONE cannot be ahead of this wait either: P_j V_j
+                // needs this warp's P_j.  The MMA that may still run now is
+                // S_{j+1}, into the other S/P buffer.
                 ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
