@@ -27,6 +27,9 @@
  * Conventions for every call below:
  *   - Device pointers are caller-owned (the library never allocates or frees
  *     device memory and never synchronises the device inside compute calls).
+ *     One exception: a fixed PKV_STATIC_WORKSPACE_BYTES (16 MiB) array in
+ *     device memory on every GPU that loads the library, used only by
+ *     pkv_paged_attention_decode_static_workspace (declared below).
  *     Tensors are dense and row-major in the shapes given; K/V/query/output
  *     pointers must be 16-byte aligned.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
@@ -134,7 +137,8 @@ pkv_status pkv_kv_cache_write(const void *key, const void *value,
  * swap-out to host and swap-in.  block_bytes = block_size * num_kv_heads *
  * head_dim * 2, a multiple of 16 (else PKV_ERR_UNSUPPORTED).  Destination
  * blocks must be distinct and not also sources in the same call.  num_pairs
- * is at most 2^30 (one CTA per pair and K or V; else PKV_ERR_UNSUPPORTED);
+ * is below 2^30 (two CTAs per pair, one for K and one for V, and a grid holds
+ * fewer than 2^31; else PKV_ERR_UNSUPPORTED);
  * caches 16-byte aligned and the mapping 8-byte aligned (else
  * PKV_ERR_MISALIGNED).  Out-of-range pairs are skipped and set
  * PKV_DEVFLAG_BLOCK_RANGE.
@@ -274,6 +278,19 @@ pkv_status pkv_paged_attention_decode_cascade(
     pkv_dtype dtype, void *stream);
 
 /*
+ * hbm_read_probe -- measurement only (the pages have no counterpart): reads
+ * `bytes` of device memory at `buf` once, with 16-byte loads that bypass L1,
+ * and folds them into *sink (device memory, 4-byte aligned; its value has no
+ * meaning).  A read-only stream is the bound of a kernel that mostly reads,
+ * such as decode attention; the benchmark times this call to report the
+ * decode kernels' fraction of it next to the copy peak.  `grid` CTAs of 512
+ * threads.  buf 16-byte aligned and bytes a multiple of 16 (else
+ * PKV_ERR_MISALIGNED / PKV_ERR_INVALID_ARG).  Asynchronous on `stream`.
+ */
+pkv_status pkv_hbm_read_probe(const void *buf, size_t bytes, unsigned int *sink, int grid,
+                              void *stream);
+
+/*
  * paged_attention_decode_static_workspace -- the same decode as
  * pkv_paged_attention_decode, for callers that cannot allocate device memory
  * at call time (an allocator that owns the whole pool, a serving runtime that
@@ -286,7 +303,10 @@ pkv_status pkv_paged_attention_decode_cascade(
  * on every GPU that loads it, until the process exits; nothing is allocated
  * per call.  The first call on a device looks up that array's device address
  * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  All calls share the one array, which keeps the
+ * before any stream capture.  The address is remembered per device and
+ * context: after cudaDeviceReset (a new context, the module loaded again) the
+ * next call looks it up again, so make that call before any capture as well.
+ * All calls share the one array, which keeps the
  * last call's contents (no part of it needs to start at zero): calls whose
  * kernels overlap on the GPU race and must be serialised by the caller.  A
  * plan needing more than PKV_STATIC_WORKSPACE_BYTES returns

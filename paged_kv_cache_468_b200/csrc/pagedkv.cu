@@ -327,8 +327,8 @@ pkv_status pkv_copy_blocks(const void *src_key_cache, const void *src_value_cach
     if (block_bytes % 16 != 0)
         return fail(PKV_ERR_UNSUPPORTED, "block_bytes %lld is not a multiple of 16",
                     (long long)block_bytes);
-    if (num_pairs > (1 << 30))
-        return fail(PKV_ERR_UNSUPPORTED, "num_pairs %d > 2^30", num_pairs);
+    if (num_pairs >= (1 << 30))   // 2 CTAs per pair must fit gridDim.x (< 2^31)
+        return fail(PKV_ERR_UNSUPPORTED, "num_pairs %d >= 2^30", num_pairs);
     if (num_pairs == 0)
         return PKV_OK;
     if (!src_key_cache || !src_value_cache || !dst_key_cache || !dst_value_cache || !block_mapping)
@@ -834,24 +834,64 @@ namespace {
 constexpr size_t kStaticWorkspaceBytes = PKV_STATIC_WORKSPACE_BYTES;
 static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
-// Device address of g_static_workspace on `dev`, looked up once per device
-// with that device current.  In host code the symbol is only a stand-in for
-// the device array, so its address must come from cudaGetSymbolAddress.
+// The current context's unique id (cuCtxGetId), or 0 when there is no
+// current context or the driver does not offer the call.  Ids are never
+// reused within a process, unlike context handles.
+unsigned long long current_context_id()
+{
+    using GetCurrentFn = CUresult (*)(CUcontext *);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+    static GetCurrentFn get_current = nullptr;
+    static GetIdFn get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrentFn>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetIdFn>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
+}
+
+// Device address of g_static_workspace in the current context of `dev`.  In
+// host code the symbol is only a stand-in for the device array, so its
+// address comes from cudaGetSymbolAddress, called with that device current.
+// The address is kept per device together with the id of the context it was
+// looked up in: a new context on the device (after cudaDeviceReset, say)
+// reloads the module, and the next call looks the address up again.
 pkv_status static_workspace_ptr(int dev, void **ptr)
 {
-    static void *cache[64] = {};
+    struct Entry {
+        unsigned long long ctx;
+        void *addr;
+    };
+    static Entry cache[64] = {};
     static std::mutex mu;
     std::lock_guard<std::mutex> lk(mu);
-    if (dev >= 0 && dev < 64 && cache[dev]) {
-        *ptr = cache[dev];
+    const bool slot = dev >= 0 && dev < 64;
+    const unsigned long long id = current_context_id();
+    if (slot && id != 0 && cache[dev].addr && cache[dev].ctx == id) {
+        *ptr = cache[dev].addr;
         return PKV_OK;
     }
     void *p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess)
         return cuda_fail(e, "cudaGetSymbolAddress(static workspace)");
-    if (dev >= 0 && dev < 64)
-        cache[dev] = p;
+    // the lookup made the device's primary context current if none was
+    const unsigned long long now = current_context_id();
+    if (slot && now != 0)
+        cache[dev] = Entry{now, p};
     *ptr = p;
     return PKV_OK;
 }

@@ -171,7 +171,18 @@ def test_copy_blocks_host_validation():
     assert call(sb=0) == pagedkv.ERR_INVALID_ARG
     assert call(bb=24) == pagedkv.ERR_UNSUPPORTED                   # not a multiple of 16
     assert call(n=(1 << 30) + 1) == pagedkv.ERR_UNSUPPORTED         # grid of 2 CTAs per pair
+    assert call(n=1 << 30) == pagedkv.ERR_UNSUPPORTED               # 2^31 CTAs: one too many
     assert call(n=0, p=None, m=None) == pagedkv.OK
     assert call(m=None) == pagedkv.ERR_INVALID_ARG
     assert call(p=a16 + 8) == pagedkv.ERR_MISALIGNED
     assert call(m=a16 + 4) == pagedkv.ERR_MISALIGNED
+
+
+def test_hbm_read_probe_host_validation():
+    L = pkv.lib()
+    a16 = 0x10000
+    assert L.pkv_hbm_read_probe(None, 16, a16, 1, None) == pagedkv.ERR_INVALID_ARG
+    assert L.pkv_hbm_read_probe(a16, 24, a16, 1, None) == pagedkv.ERR_INVALID_ARG   # not 16-byte units
+    assert L.pkv_hbm_read_probe(a16, 16, a16, 0, None) == pagedkv.ERR_INVALID_ARG   # empty grid
+    assert L.pkv_hbm_read_probe(a16 + 8, 16, a16, 1, None) == pagedkv.ERR_MISALIGNED
+    assert L.pkv_hbm_read_probe(a16, 16, a16 + 2, 1, None) == pagedkv.ERR_MISALIGNED

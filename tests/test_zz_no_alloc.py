@@ -2,10 +2,13 @@
 
 pkv_paged_attention_decode_static_workspace takes its split-plan workspace
 from a fixed array the library reserves on each GPU, so nothing is allocated
-when it runs.  This test calls it through the C ABI twice in a row, on two
-different split workloads (the second call reuses the array the first one
-left behind), and checks each output against the regular entry point with a
-caller-provided workspace, within the parity tolerance of the other tests.
+when it runs.  Such callers include a serving runtime whose allocator owns the
+whole device pool, or plain C code that has no device allocator at hand.  The
+tests call it through the C ABI several times in a row, on different split
+workloads (each call reuses the array the previous one left behind), and
+check that every output equals, bit for bit, the regular entry point's with a
+caller-provided workspace: both run the same kernels on the same plan.  One
+plan needs the whole array but 16 bytes; one sequence more is refused.
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test; it also passes alone in a fresh process.
@@ -17,7 +20,7 @@ import torch
 
 import paged_kv_cache_468_b200 as pkv
 from paged_kv_cache_468_b200 import pagedkv, workloads
-from tests.parity_util import TOL
+from tests.parity_util import custom
 
 pytestmark = pytest.mark.gpu
 
@@ -48,6 +51,33 @@ def _static_call(f, d, partition_tokens):
     return out
 
 
+def _regular_call(d, partition_tokens):
+    return pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"],
+                                      d["block_tables"], d["context_lens"], d["scale"],
+                                      partition_tokens=partition_tokens)
+
+
+def _need(d, partition_tokens):
+    B, Hq, D = d["query"].shape
+    NB, bs, Hkv, _ = d["key_cache"].shape
+    return pkv.decode_workspace_bytes(B, Hq, Hkv, D, d["block_tables"].shape[1], bs,
+                                      partition_tokens)
+
+
+# 205 sequences x 10 query heads x 31 partitions x (64 + 2) floats: 16 bytes
+# short of the 16 MiB array (records of (D + 2) * 4 bytes never fill it exactly)
+_NEAR_CAP = dict(B=205, Hq=10, Hkv=2, D=64, bs=16, pt=32, span=992)
+
+
+def _near_cap_inputs(batch):
+    c = _NEAR_CAP
+    g = torch.Generator().manual_seed(31)
+    lens = torch.randint(1, c["span"] + 1, (batch,), generator=g).tolist()
+    lens[0] = c["span"]                              # 62 blocks: 31 partitions of 32 tokens
+    step = custom("near_cap", batch, c["Hq"], c["Hkv"], c["D"], c["bs"], "bf16", lens, seed=32)
+    return {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
+
+
 def test_static_workspace_matches_regular_entry_twice_in_a_row():
     f = _entry()
     cases = [
@@ -57,16 +87,32 @@ def test_static_workspace_matches_regular_entry_twice_in_a_row():
     pkv.device_flags(clear=True)
     for cfg, batch, pt in cases:
         d = _inputs(cfg, batch)
-        B, Hq, D = d["query"].shape
-        NB, bs, Hkv, _ = d["key_cache"].shape
-        assert pkv.decode_workspace_bytes(B, Hq, Hkv, D, d["block_tables"].shape[1], bs, pt) > 0
-        ref = pkv.paged_attention_decode(d["query"], d["key_cache"], d["value_cache"],
-                                         d["block_tables"], d["context_lens"], d["scale"],
-                                         partition_tokens=pt)
+        assert _need(d, pt) > 0
+        ref = _regular_call(d, pt)
         got = _static_call(f, d, pt)
         torch.cuda.synchronize()
-        err = (got.float() - ref.float()).abs().max().item()
-        assert err <= TOL[cfg.dtype], (cfg.name, err)
+        assert torch.equal(got, ref), (cfg.name, (got.float() - ref.float()).abs().max().item())
+    assert pkv.device_flags() == 0
+
+
+def test_static_workspace_plan_that_fills_the_array():
+    f = _entry()
+    c = _NEAR_CAP
+    pkv.device_flags(clear=True)
+    # a first call leaves other records in the array
+    d0 = _inputs(workloads.CONFIGS["long_split"], 2)
+    first = _static_call(f, d0, 512)
+    assert torch.equal(first, _regular_call(d0, 512))
+    d = _near_cap_inputs(c["B"])
+    need = _need(d, c["pt"])
+    assert pkv.decode_plan(c["B"], c["Hq"], c["Hkv"], c["D"], d["block_tables"].shape[1], c["bs"],
+                           c["pt"]) == (c["pt"], 31)
+    assert need == c["B"] * c["Hq"] * 31 * (c["D"] + 2) * 4 == (16 << 20) - 16
+    ref = _regular_call(d, c["pt"])
+    for _ in range(2):                                # twice: the second reuses the first's records
+        got = _static_call(f, d, c["pt"])
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref), (got.float() - ref.float()).abs().max().item()
     assert pkv.device_flags() == 0
 
 
@@ -77,3 +123,8 @@ def test_static_workspace_rejects_plans_beyond_its_size():
            pagedkv.BF16, None)
     assert st == pagedkv.ERR_WORKSPACE
     assert "static workspace" in pkv.lib().pkv_last_error().decode()
+    # one sequence more than the plan that fills the array is refused, before any launch
+    c = _NEAR_CAP
+    st = f(None, None, None, None, c["span"] // c["bs"], None, c["B"] + 1, c["Hq"], c["Hkv"], c["D"],
+           c["bs"], 1 << 16, 0.125, c["pt"], None, pagedkv.BF16, None)
+    assert st == pagedkv.ERR_WORKSPACE
