@@ -173,24 +173,27 @@ def committed_traffic(config_name: str, split: bool, cascade: bool):
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    """nvidia-smi clock / throttle-reason samples taken while timed regions run.
+
+    The sampler runs for the whole measurement; mark(True) / mark(False)
+    bracket each timed region, and only samples inside a region count."""
 
     FIELDS = ["clocks.sm", "clocks.max.sm", "clocks_event_reasons.hw_slowdown",
               "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
               "clocks_event_reasons.sw_power_cap"]
+    PERIOD_MS = 50
 
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
         self.lines = []
-        self.t_on = None
-        self.t_off = None
+        self.windows = []          # [t_on, t_off] per timed region
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + ",".join(self.FIELDS),
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
@@ -207,13 +210,17 @@ class ClockSampler:
 
     def mark(self, on: bool):
         if on:
-            self.t_on = time.time()
-        else:
-            self.t_off = time.time()
+            self.windows.append([time.time(), None])
+        elif self.windows and self.windows[-1][1] is None:
+            self.windows[-1][1] = time.time()
+
+    def _inside(self, t: float) -> bool:
+        return any(a <= t <= (b if b is not None else float("inf")) + 0.06 for a, b in self.windows)
 
     def stop(self) -> dict:
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
         time.sleep(0.12)
         self.proc.terminate()
         try:
@@ -222,22 +229,20 @@ class ClockSampler:
             self.proc.kill()
         rows = []
         for t, line in self.lines:
-            if self.t_on is not None and self.t_off is not None and not (self.t_on <= t <= self.t_off + 0.06):
+            if not self._inside(t):
                 continue
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            rows.append(parts)
-        if not rows:   # timed region shorter than the sampling period: take the nearest
-            rows = [[p.strip() for p in l.split(",")] for _, l in self.lines[-3:]]
-            rows = [r for r in rows if len(r) == len(self.FIELDS)]
+            if len(parts) == len(self.FIELDS):
+                rows.append(parts)
         sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
         mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[2 + i].lower() == "active"})
+        timed_s = sum((b or a) - a for a, b in self.windows)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "period_ms": self.PERIOD_MS,
+                "timed_regions": len(self.windows), "timed_s": round(timed_s, 3)}
 
 
 def dist_setup():
@@ -334,12 +339,41 @@ def choose_oracle_seqs(step, cfg, nthreads, budget_s):
     return max(1, min(B, int(budget_s / max(el, 1e-6))))
 
 
+L2_BYTES_B200 = 126 << 20     # the B200's L2; workloads whose K/V fit get an L2 flush per iteration
+
+
+def fits_in_l2(nbytes: dict, l2_bytes: int = L2_BYTES_B200) -> bool:
+    return nbytes["kv_unique"] <= l2_bytes
+
+
+def workload_config(cfg, step: dict, nbytes: dict, world: int) -> dict:
+    """The `config` object of a JSON line: the workload and how it is timed.
+    Both arms (GPU and reference) print the same one for the same workload."""
+    B, Hq, D = step["query"].shape
+    NB, bs, Hkv, _ = step["key_cache"].shape
+    l2_mib = L2_BYTES_B200 >> 20
+    if fits_in_l2(nbytes):
+        l2 = (f"inputs fit in L2 ({nbytes['kv_unique'] / 1e6:.1f} MB of K/V vs {l2_mib} MiB): each "
+              f"timed iteration has its own CUDA events and a {2 * l2_mib} MiB buffer is written "
+              f"between iterations, outside the events")
+    else:
+        l2 = (f"inputs larger than L2: {nbytes['kv_unique'] / 1e6:.0f} MB of K/V per step vs "
+              f"{l2_mib} MiB L2, no flush")
+    return {"workload": cfg.name, "description": cfg.description, "batch": int(B),
+            "num_heads": int(Hq), "num_kv_heads": int(Hkv), "head_dim": int(D),
+            "block_size": int(bs), "num_blocks": int(NB),
+            "max_blocks": int(step["block_tables"].shape[1]),
+            "context_tokens": int(nbytes["kv_tokens"]), "kv_dtype": cfg.dtype,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU", "l2": l2}
+
+
 def run_reference(args, cfg, world, rank):
     """The oracle as the reference arm (rank 0 only)."""
     if rank != 0:
         return 0
     nthreads = os.cpu_count() or 1
-    step = workloads.make_decode_step(cfg)
+    step = workloads.make_decode_step(dataclass_replace(cfg, seed=replica_seed(cfg.seed, 0)))
+    nbytes = step_bytes(step, cfg)
     total_budget = args.reference_seconds
     per_step = total_budget / max(1, args.steps + args.warmup)
     nseq = choose_oracle_seqs(step, cfg, nthreads, per_step)
@@ -358,7 +392,7 @@ def run_reference(args, cfg, world, rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * t_total / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": cfg.name, "description": cfg.description},
+        "config": workload_config(cfg, step, nbytes, world),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": nthreads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -370,61 +404,298 @@ def run_reference(args, cfg, world, rank):
 
 # ------------------------------------------------------------- GPU arm ----
 
+def time_back_to_back(fn, n: int, stream) -> float:
+    """ms per call of fn over n calls issued back to back: one CUDA event pair
+    on the launching stream around all of them."""
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(n):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / n
+
+
+def time_each(fn, n: int, stream, flush_buf=None) -> list:
+    """ms of each of n calls (an event pair around each); with flush_buf, a
+    write of that buffer between calls, outside the events, so no call reads
+    data an earlier one left in L2."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    torch.cuda.synchronize()
+    for i in range(n):
+        if flush_buf is not None:
+            flush_buf.fill_(i & 0xff)
+        evs[i][0].record(stream)
+        fn()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    return [x.elapsed_time(y) for x, y in evs]
+
+
+class DecodeWorkload:
+    """One workload resident on the GPU: its step inputs, the decode call
+    (plain or cascade) and the step (slot_mapping write + decode)."""
+
+    def __init__(self, pkv, cfg, dev, seed: int, partition_tokens, cascade_mode: str):
+        self.pkv, self.cfg, self.dev = pkv, cfg, dev
+        self.step = workloads.make_decode_step(dataclass_replace(cfg, seed=seed))
+        self.nbytes = step_bytes(self.step, cfg)
+        d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in self.step.items()}
+        self.d = d
+        B, Hq, D = d["query"].shape
+        NB, bs, Hkv, _ = d["key_cache"].shape
+        MB = d["block_tables"].shape[1]
+        self.B = int(B)
+        self.pt_req = cfg.partition_tokens if partition_tokens is None else partition_tokens
+        self.plan_pt, self.plan_np = pkv.decode_plan(B, Hq, Hkv, D, MB, bs, self.pt_req)
+        self.cascade = cascade_mode == "on" or (cascade_mode == "auto" and cfg.shared_prefix > 0)
+        ws_bytes = pkv.decode_workspace_bytes(B, Hq, Hkv, D, MB, bs, self.pt_req)
+        self.launches_per_step = 2 + (1 if self.plan_np > 1 else 0)
+        self.cas = None
+        if self.cascade:
+            self.cas = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in
+                        workloads.cascade_inputs(self.step, cfg.shared_prefix, cfg.samples).items()}
+            ws_bytes = int(pkv.lib().pkv_decode_cascade_workspace_bytes(
+                B, Hq, Hkv, D, self.cas["prefix_tables"].shape[1], self.cas["suffix_tables"].shape[1],
+                self.cas["max_group_size"], bs, self.pt_req))
+            self.launches_per_step = 4
+        self.ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
+        self.out = torch.empty_like(d["query"])
+        self.flush = fits_in_l2(self.nbytes)
+
+    # the tensors a caller supplies every step (the rest stays resident: the pool)
+    def step_input_names(self) -> list:
+        names = ["query", "new_key", "new_value", "slot_mapping"]
+        if self.cascade:
+            return names + ["prefix_tables", "prefix_lens", "group_start", "suffix_tables",
+                            "suffix_lens"]
+        return names + ["block_tables", "context_lens"]
+
+    def step_inputs(self) -> dict:
+        src = dict(self.d)
+        if self.cascade:
+            src.update({k: v for k, v in self.cas.items() if isinstance(v, torch.Tensor)})
+        return {k: src[k] for k in self.step_input_names()}
+
+    def decode(self, x: dict = None, out=None):
+        x = self.step_inputs() if x is None else x
+        out = self.out if out is None else out
+        d, pkv = self.d, self.pkv
+        if self.cascade:
+            return pkv.paged_attention_decode_cascade(
+                x["query"], d["key_cache"], d["value_cache"], x["prefix_tables"], x["prefix_lens"],
+                x["group_start"], x["suffix_tables"], x["suffix_lens"], d["scale"],
+                max_group_size=self.cas["max_group_size"], partition_tokens=self.pt_req, out=out,
+                workspace=self.ws)
+        return pkv.paged_attention_decode(x["query"], d["key_cache"], d["value_cache"],
+                                          x["block_tables"], x["context_lens"], d["scale"],
+                                          partition_tokens=self.pt_req, out=out, workspace=self.ws)
+
+    def write(self, x: dict = None):
+        x = self.step_inputs() if x is None else x
+        self.pkv.kv_cache_write(x["new_key"], x["new_value"], x["slot_mapping"], self.d["key_cache"],
+                                self.d["value_cache"])
+
+    def one_step(self):
+        self.write()
+        self.decode()
+
+    def kernel_name(self) -> str:
+        if self.cascade:
+            return "prefix_tc_kernel + paged_decode_kernel (suffixes) + lse_merge_cascade_kernel"
+        return "paged_decode_kernel" + (" + lse_merge_kernel" if self.plan_np > 1 else "")
+
+    def traffic(self):
+        return committed_traffic(self.cfg.name, self.plan_np > 1 and not self.cascade, self.cascade)
+
+    def method(self) -> dict:
+        return {"partition_tokens": self.plan_pt, "num_partitions": self.plan_np,
+                "cascade": self.cascade}
+
+
+def measure_decode_launches(w: DecodeWorkload, n: int, stream, flush_buf, sampler=None) -> dict:
+    """The decode call alone, n launches: the mean from one event pair around
+    back-to-back launches (per-launch events with an L2 flush in between for
+    workloads that fit in L2) and the spread from per-launch events."""
+    for _ in range(3):
+        w.decode()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.mark(True)
+    if w.flush:
+        each = time_each(w.decode, n, stream, flush_buf)
+        mean = statistics.mean(each)
+        timing = (f"{n} launches, an event pair around each, a {flush_buf.numel() >> 20} MiB "
+                  f"L2 flush between them")
+    else:
+        mean = time_back_to_back(w.decode, n, stream)
+        each = time_each(w.decode, min(n, 2000), stream)
+        timing = f"mean: one event pair around {n} back-to-back launches; spread: per-launch events"
+    if sampler:
+        sampler.mark(False)
+    q = statistics.quantiles(each, n=10) if len(each) >= 10 else [min(each)] * 9
+    return {"mean_ms": mean, "median_ms": statistics.median(each), "p10_ms": q[0],
+            "p90_ms": q[-1], "n": n, "timing": timing}
+
+
+def read_ceiling(pkv, dev, stream, nbytes: int = 2 << 30, reps: int = 40) -> dict:
+    """Read-only HBM streaming rate (16-byte loads over nbytes), best over a
+    few grid sizes: the ceiling of a kernel that only reads."""
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    buf.fill_(1)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    rates = {}
+    for per_sm in (2, 4, 8):
+        grid = sms * per_sm
+        fn = lambda: pkv.hbm_read_probe(buf, sink, grid)
+        for _ in range(3):
+            fn()
+        ms = time_back_to_back(fn, reps, stream)
+        rates[str(grid)] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+    del buf
+    return {"gbs": max(rates.values()), "bytes": nbytes, "reps": reps, "by_grid": rates,
+            "kernel": "hbm_read_probe_kernel (16-byte ld.global.nc, 8 in flight per thread)"}
+
+
+def roofline_entry(w: DecodeWorkload, t: dict, peaks: dict, ceiling) -> dict:
+    bytes_ = w.nbytes["decode_unique"]
+    achieved = bytes_ / (t["mean_ms"] * 1e-3) / 1e9
+    r = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+         "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": w.traffic(),
+         "peak_source": (peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, a copy: read + write)"
+                         if peaks["source"] == "measured" else "fallback 6650 GB/s (copy)"),
+         "kernel": w.kernel_name(), "bytes_per_launch": bytes_,
+         "launch_ms": round(t["mean_ms"], 5), "launch_ms_median": round(t["median_ms"], 5),
+         "launch_ms_p10": round(t["p10_ms"], 5), "launch_ms_p90": round(t["p90_ms"], 5),
+         "launches_timed": t["n"], "timing": t["timing"],
+         "frac_median": round(bytes_ / (t["median_ms"] * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+         "frac_of_8000": round(achieved / 8000.0, 4)}
+    if ceiling:
+        r["read_ceiling_gbs"] = ceiling["gbs"]
+        r["frac_of_read_ceiling"] = round(achieved / ceiling["gbs"], 4)
+    return r
+
+
+def per_config_entry(w: DecodeWorkload, t: dict, peaks: dict, ceiling) -> dict:
+    ms = t["mean_ms"]
+    nb = w.nbytes
+    e = {"decode_ms": round(ms, 5), "seq_per_s": round(w.B / (ms * 1e-3), 1),
+         "tokens_per_s": round(w.B / (ms * 1e-3), 1),
+         "kv_tokens_per_s": round(nb["kv_tokens"] / (ms * 1e-3), 1),
+         "kv_gbs_unique": round(nb["kv_unique"] / (ms * 1e-3) / 1e9, 1),
+         "kv_gbs_logical": round(nb["kv"] / (ms * 1e-3) / 1e9, 1),
+         "method": w.method(), "roofline": roofline_entry(w, t, peaks, ceiling)}
+    if nb["kv_unique"] != nb["kv"]:
+        e["bytes_unique"], e["bytes_logical"] = nb["decode_unique"], nb["decode"]
+    return e
+
+
+def e2e_pipelined(w: DecodeWorkload, steps: int, warmup: int, dev) -> dict:
+    """The step end to end through the public calls, with host buffers: every
+    step copies its inputs from pinned host memory and its output back.  Two
+    sets of device buffers and two copy streams let step i+1's inputs travel
+    while step i computes and step i-1's output returns; the caller reads
+    step i-1's output while step i runs."""
+    host_in = {k: v.cpu().pin_memory() for k, v in w.step_inputs().items()}
+    host_out = [torch.empty(w.out.shape, dtype=w.out.dtype).pin_memory() for _ in range(2)]
+    dev_in = [{k: torch.empty_like(v, device=dev) for k, v in host_in.items()} for _ in range(2)]
+    outs = [torch.empty_like(w.out) for _ in range(2)]
+    comp = torch.cuda.current_stream(dev)
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = host_out[0].numel() * host_out[0].element_size()
+
+    def run(n):
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(up)
+        checksum = 0.0
+        for i in range(n):
+            s = i & 1
+            with torch.cuda.stream(up):
+                if i >= 2:
+                    up.wait_event(comp_done[s])          # step i-2 has read buffer set s
+                for k, v in host_in.items():
+                    dev_in[s][k].copy_(v, non_blocking=True)
+                h2d_done[s].record(up)
+            comp.wait_event(h2d_done[s])
+            w.write(dev_in[s])
+            w.decode(dev_in[s], out=outs[s])
+            comp_done[s].record(comp)
+            with torch.cuda.stream(down):
+                down.wait_event(comp_done[s])
+                host_out[s].copy_(outs[s], non_blocking=True)
+                d2h_done[s].record(down)
+            if i >= 1:                                   # the caller reads step i-1's result
+                d2h_done[(i - 1) & 1].synchronize()
+                checksum += float(host_out[(i - 1) & 1][0, 0, 0])
+        down.wait_stream(comp)
+        end.record(down)
+        end.synchronize()
+        checksum += float(host_out[(n - 1) & 1][0, 0, 0])
+        return start.elapsed_time(end) / n
+
+    run(max(3, warmup))
+    ms = run(steps)
+    return {"ms": ms, "h2d": h2d, "d2h": d2h,
+            "mode": "pipelined: two device buffer sets, inputs up and outputs down on two copy "
+                    "streams, overlapping the previous and next steps' kernels"}
+
+
+def e2e_serial(w: DecodeWorkload, steps: int, warmup: int, dev, flush_buf) -> dict:
+    """As e2e_pipelined, one step at a time (each synchronised), for workloads
+    that fit in L2: an L2 flush between steps, outside the events."""
+    host_in = {k: v.cpu().pin_memory() for k, v in w.step_inputs().items()}
+    host_out = torch.empty(w.out.shape, dtype=w.out.dtype).pin_memory()
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        for k, v in host_in.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        w.write(dev_in)
+        w.decode(dev_in)
+        host_out.copy_(w.out, non_blocking=True)
+        stream.synchronize()                            # the caller reads the result
+
+    for _ in range(max(3, warmup)):
+        one()
+    each = time_each(one, steps, stream, flush_buf)
+    return {"ms": statistics.mean(each), "h2d": sum(t.numel() * t.element_size() for t in host_in.values()),
+            "d2h": host_out.numel() * host_out.element_size(),
+            "mode": "serial: one step at a time, L2 flushed between steps"}
+
+
 def run_gpu(args, cfg, world, rank, local):
     import paged_kv_cache_468_b200 as pkv
 
     dev = torch.device("cuda", local)
-    step = workloads.make_decode_step(dataclass_replace(cfg, seed=replica_seed(cfg.seed, rank)))
-    nbytes = step_bytes(step, cfg)
-    d = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
-    B, Hq, D = d["query"].shape
-    NB, bs, Hkv, _ = d["key_cache"].shape
-    MB = d["block_tables"].shape[1]
-    pt_req = cfg.partition_tokens if args.partition_tokens is None else args.partition_tokens
-    plan_pt, plan_np = pkv.decode_plan(B, Hq, Hkv, D, MB, bs, pt_req)
-    ws_bytes = pkv.decode_workspace_bytes(B, Hq, Hkv, D, MB, bs, pt_req)
-    out = torch.empty_like(d["query"])
-    launches_per_step = 2 + (1 if plan_np > 1 else 0)
     stream = torch.cuda.current_stream(dev)
-    cascade = args.cascade == "on" or (args.cascade == "auto" and cfg.shared_prefix > 0)
-    if cascade:
-        cas = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in
-               workloads.cascade_inputs(step, cfg.shared_prefix, cfg.samples).items()}
-        ws_bytes = int(pkv.lib().pkv_decode_cascade_workspace_bytes(
-            B, Hq, Hkv, D, cas["prefix_tables"].shape[1], cas["suffix_tables"].shape[1],
-            cas["max_group_size"], bs, pt_req))
-        launches_per_step = 4
-    ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
-
-    def decode_call(query, tables, lens):
-        if cascade:
-            return pkv.paged_attention_decode_cascade(
-                query, d["key_cache"], d["value_cache"], cas["prefix_tables"], cas["prefix_lens"],
-                cas["group_start"], cas["suffix_tables"], cas["suffix_lens"], d["scale"],
-                max_group_size=cas["max_group_size"], partition_tokens=pt_req, out=out,
-                workspace=ws)
-        return pkv.paged_attention_decode(query, d["key_cache"], d["value_cache"], tables, lens,
-                                          d["scale"], partition_tokens=pt_req, out=out,
-                                          workspace=ws)
-
-    def one_step():
-        pkv.kv_cache_write(d["new_key"], d["new_value"], d["slot_mapping"], d["key_cache"],
-                           d["value_cache"])
-        decode_call(d["query"], d["block_tables"], d["context_lens"])
+    w = DecodeWorkload(pkv, cfg, dev, replica_seed(cfg.seed, rank), args.partition_tokens,
+                       args.cascade)
+    nbytes = w.nbytes
+    l2_dev = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or 0)
+    flush_buf = torch.empty(2 * max(l2_dev, L2_BYTES_B200), dtype=torch.uint8, device=dev)
 
     pkv.device_flags(clear=True)
     for _ in range(args.warmup):
-        one_step()
+        w.one_step()
     torch.cuda.synchronize()
 
     # optional: the step as a CUDA graph (same kernels, no per-launch host work)
-    step_fn = one_step
+    step_fn = w.one_step
     graph_note = "off"
     if args.graph:
         try:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph):
-                one_step()
+                w.one_step()
             for _ in range(3):
                 graph.replay()
             torch.cuda.synchronize()
@@ -434,37 +705,7 @@ def run_gpu(args, cfg, world, rank, local):
             graph_note = f"capture failed ({type(exc).__name__}); plain launches"
             torch.cuda.synchronize()
 
-    # ---- L2: inputs that fit in L2 would be read warm from the second
-    # iteration on; for those, every timed iteration gets its own events and a
-    # write of twice the L2 size in between (outside the events) ----
-    l2_bytes = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 126 << 20) or (126 << 20))
-    flush_l2 = nbytes["kv_unique"] <= l2_bytes
-    flush_buf = torch.empty(2 * l2_bytes, dtype=torch.uint8, device=dev) if flush_l2 else None
-
-    def timed_iterations(fn, n):
-        """ms per iteration of fn over n iterations: one event pair around all
-        of them, or (inputs fitting in L2) per iteration with an L2 flush
-        between iterations; also the per-iteration times when taken."""
-        if not flush_l2:
-            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record(stream)
-            for _ in range(n):
-                fn()
-            b_.record(stream)
-            torch.cuda.synchronize()
-            return a.elapsed_time(b_) / n, None
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(n)]
-        for i in range(n):
-            flush_buf.fill_(i & 0xff)
-            evs[i][0].record(stream)
-            fn()
-            evs[i][1].record(stream)
-        torch.cuda.synchronize()
-        per = [x.elapsed_time(y) for x, y in evs]
-        return sum(per) / n, per
-
-    # ---- device-timed region (inputs resident in HBM): K whole steps ----
+    # ---- the contract's timed region: K whole steps, inputs resident in HBM ----
     K = args.steps
     sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
     if sampler:
@@ -473,121 +714,101 @@ def run_gpu(args, cfg, world, rank, local):
     torch.cuda.synchronize()
     if sampler:
         sampler.mark(True)
-    ms_step_mean, _ = timed_iterations(step_fn, K)
+    if w.flush:
+        ms_step_local = statistics.mean(time_each(step_fn, K, stream, flush_buf))
+    else:
+        ms_step_local = time_back_to_back(step_fn, K, stream)
     if sampler:
         sampler.mark(False)
     barrier(world)
-    ms_total = ms_step_mean * K
-    clocks = sampler.stop() if sampler else None
 
-    # ---- the decode call alone (its kernels), for the roofline: CUDA events
-    # around each launch on the launching stream ----
-    Kd = max(1, min(K, args.roofline_launches))
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(Kd)]
-    torch.cuda.synchronize()
-    for i in range(Kd):
-        if flush_l2:
-            flush_buf.fill_(i & 0xff)
-        ev[i][0].record(stream)
-        decode_call(d["query"], d["block_tables"], d["context_lens"])
-        ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    decode_times = [a.elapsed_time(b) for a, b in ev]
-    decode_ms = statistics.mean(decode_times)      # decode (+ merge) per call
-    decode_ms_median = statistics.median(decode_times)
+    # ---- the decode call alone, for the roofline: at least --roofline-launches
+    # launches and --roofline-seconds of device time, whatever --steps is ----
+    n_roof = max(args.roofline_launches,
+                 int(math.ceil(args.roofline_seconds * 1e3 / max(ms_step_local, 1e-4))))
+    n_roof = min(n_roof, 50000)
+    t_main = measure_decode_launches(w, n_roof, stream, flush_buf, sampler)
     flags = pkv.device_flags(clear=True)
 
     # ---- end to end through the public API, host buffers ----
     e2e = None
     if not args.no_e2e:
-        host_in = {k: d[k].cpu().pin_memory() for k in
-                   ("query", "new_key", "new_value", "slot_mapping", "block_tables", "context_lens")}
-        host_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-        d2h = host_out.numel() * host_out.element_size()
-        dev_in = {k: torch.empty_like(v, device=dev) for k, v in host_in.items()}
-
-        def e2e_step():
-            for k, v in host_in.items():
-                dev_in[k].copy_(v, non_blocking=True)
-            pkv.kv_cache_write(dev_in["new_key"], dev_in["new_value"], dev_in["slot_mapping"],
-                               d["key_cache"], d["value_cache"])
-            decode_call(dev_in["query"], dev_in["block_tables"], dev_in["context_lens"])
-            host_out.copy_(out, non_blocking=True)
-            stream.synchronize()                       # the caller reads the result
-
-        for _ in range(max(3, args.warmup)):
-            e2e_step()
-        Ke = max(1, min(K, args.e2e_steps))
+        Ke = max(1, min(K, args.e2e_steps)) if w.flush else max(K, args.e2e_steps)
         barrier(world)
-        torch.cuda.synchronize()
-        e2e_local, _ = timed_iterations(e2e_step, Ke)
+        r = e2e_serial(w, Ke, args.warmup, dev, flush_buf) if w.flush else \
+            e2e_pipelined(w, Ke, args.warmup, dev)
         barrier(world)
-        e2e_ms = max_over_ranks(e2e_local, world)
+        e2e_ms = max_over_ranks(r["ms"], world)
         e2e_gbs = sum_over_ranks(nbytes["decode_unique"] + nbytes["write"], world) / (e2e_ms * 1e-3) / 1e9
-        e2e = {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4), "steps": Ke,
-               "tokens_per_s": round(sum_over_ranks(B, world) / (e2e_ms * 1e-3), 1)}
+        e2e = {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": r["h2d"],
+               "d2h_bytes_per_step": r["d2h"], "ms_per_step": round(e2e_ms, 4), "steps": Ke,
+               "tokens_per_s": round(sum_over_ranks(w.B, world) / (e2e_ms * 1e-3), 1),
+               "mode": r["mode"]}
 
     # unique bytes: a block shared by several sequences' tables counts once
-    value, ms_step = job_throughput(nbytes["decode_unique"] + nbytes["write"], ms_total / K, world)
+    value, ms_step = job_throughput(nbytes["decode_unique"] + nbytes["write"], ms_step_local, world)
     # every collective before any rank-0-only code: all ranks take the same steps
-    tokens = sum_over_ranks(B, world)
+    tokens = sum_over_ranks(w.B, world)
     kv_tokens_all = sum_over_ranks(nbytes["kv_tokens"], world)
     kv_all = sum_over_ranks(nbytes["kv"], world)
 
     peaks = measured_peaks()
-    achieved = nbytes["decode_unique"] / (decode_ms * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": committed_traffic(cfg.name, plan_np > 1 and not cascade, cascade),
-                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs)"
-                if peaks["source"] == "measured" else "fallback 6650 GB/s",
-                "kernel": ("prefix_tc_kernel + paged_decode_kernel (suffixes) + "
-                           "lse_merge_cascade_kernel" if cascade else
-                           "paged_decode_kernel" + (" + lse_merge_kernel" if plan_np > 1 else "")),
-                "bytes_per_launch": nbytes["decode_unique"], "launch_ms": round(decode_ms, 5),
-                "launch_ms_median": round(decode_ms_median, 5),
-                "frac_of_8000": round(achieved / 8000.0, 4)}
+    ceiling = None
+    per_config = None
+    if rank == 0 and world == 1:
+        if not args.no_read_ceiling:
+            ceiling = read_ceiling(pkv, dev, stream)
+        if not args.no_per_config:
+            per_config = {}
+            for name in workloads.CONFIGS:
+                if name == cfg.name:
+                    per_config[name] = per_config_entry(w, t_main, peaks, ceiling)
+                    continue
+                other = DecodeWorkload(pkv, workloads.CONFIGS[name], dev, replica_seed(
+                    workloads.CONFIGS[name].seed, rank), None, args.cascade)
+                for _ in range(3):
+                    other.one_step()
+                est = time_back_to_back(other.decode, 5, stream)
+                n = min(20000, max(args.per_config_launches,
+                                   int(math.ceil(args.per_config_seconds * 1e3 / max(est, 1e-4)))))
+                t = measure_decode_launches(other, n, stream, flush_buf, sampler)
+                per_config[name] = per_config_entry(other, t, peaks, ceiling)
+                del other
+                torch.cuda.empty_cache()
+            flags |= pkv.device_flags(clear=True)
+    clocks = sampler.stop() if sampler else None
+    roofline = roofline_entry(w, t_main, peaks, ceiling)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nthreads = os.cpu_count() or 1
-        nseq = choose_oracle_seqs(step, cfg, nthreads, args.cpu_seconds / 3)
-        gbs, n, reps, el = oracle_sample_rate(step, cfg, args.cpu_seconds, nthreads, max_seqs=nseq)
+        nseq = choose_oracle_seqs(w.step, cfg, nthreads, args.cpu_seconds / 3)
+        gbs, n, reps, el = oracle_sample_rate(w.step, cfg, args.cpu_seconds, nthreads, max_seqs=nseq)
         cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": nthreads, "kind": "oracle",
-               "sample": f"first {n} of {B} sequences (write + decode), {reps} repetitions "
+               "sample": f"first {n} of {w.B} sequences (write + decode), {reps} repetitions "
                          f"in {el:.1f} s, fp64"}
 
     if rank == 0:
+        method = dict(w.method(), cuda_graph=graph_note,
+                      step_timing=("an event pair around each step, L2 flushed between steps"
+                                   if w.flush else "one event pair around the K steps"))
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": cfg.dtype, "data": "synthetic",
-            "config": {"workload": cfg.name, "description": cfg.description, "batch": B,
-                       "num_heads": Hq, "num_kv_heads": Hkv, "head_dim": D, "block_size": bs,
-                       "num_blocks": NB, "max_blocks": MB,
-                       "context_tokens": nbytes["kv_tokens"],
-                       "partition_tokens": plan_pt, "num_partitions": plan_np,
-                       "cascade": cascade, "cuda_graph": graph_note,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": (f"inputs fit in L2 ({nbytes['kv_unique'] / 1e6:.1f} MB of K/V vs "
-                              f"{l2_bytes / 1e6:.0f} MB): each timed iteration has its own CUDA "
-                              f"events and a {2 * l2_bytes / 1e6:.0f} MB buffer is written between "
-                              f"iterations, outside the events")
-                       if flush_l2 else
-                       (f"inputs larger than L2: {nbytes['kv_unique'] / 1e6:.0f} MB of K/V "
-                        f"per step vs {l2_bytes / 1e6:.0f} MB L2, no flush")},
+            "config": workload_config(cfg, w.step, nbytes, world),
+            "method": method,
             "tokens_per_s": round(tokens / (ms_step * 1e-3), 1),
             "kv_tokens_per_s": round(kv_tokens_all / (ms_step * 1e-3), 1),
             "frac_of_hbm_peak": round(value / peaks["hbm_gbs"], 4),
             "logical_kv_gbs": round(kv_all / (ms_step * 1e-3) / 1e9, 1),
-            "gpu_launches": launches_per_step * K,
-            "launches_per_step": launches_per_step,
+            "gpu_launches": w.launches_per_step * K,
+            "launches_per_step": w.launches_per_step,
             "device_flags": flags,
             "roofline": roofline,
+            "read_ceiling": ceiling,
+            "per_config": per_config,
             "clocks": clocks,
             "e2e": e2e,
             "cpu_baseline": cpu,
@@ -703,7 +924,15 @@ def main(argv=None):
     ap.add_argument("--partition-tokens", type=int, default=None,
                     help="override the workload's partition request (0 auto, <0 never)")
     ap.add_argument("--e2e-steps", type=int, default=200)
-    ap.add_argument("--roofline-launches", type=int, default=500)
+    ap.add_argument("--roofline-launches", type=int, default=2000,
+                    help="decode launches timed for the roofline (at least)")
+    ap.add_argument("--roofline-seconds", type=float, default=0.6,
+                    help="device time the roofline leg covers (at least)")
+    ap.add_argument("--per-config-launches", type=int, default=1000)
+    ap.add_argument("--per-config-seconds", type=float, default=0.3)
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the roofline of the other workloads")
+    ap.add_argument("--no-read-ceiling", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-seconds", type=float, default=90.0)
     ap.add_argument("--cascade", default="auto", choices=["auto", "on", "off"],

@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.pkv_alloc_new_seq_cached.restype = i32
         L.pkv_alloc_new_seq_cached.argtypes = [P, ctypes.POINTER(ctypes.c_uint64), i32, i64, pi32,
                                                i32, pint, pint]
+        L.pkv_hbm_read_probe.restype = i32
+        L.pkv_hbm_read_probe.argtypes = [P, sz, P, i32, P]
         _lib = L
         return L
 
@@ -184,6 +186,17 @@ def selftest_bounded_wait(limit_ns: int, stream: Optional[torch.cuda.Stream] = N
     dev = torch.device("cuda", torch.cuda.current_device())
     _check(lib().pkv_selftest_bounded_wait(int(limit_ns), _stream_handle(stream, dev)),
            "pkv_selftest_bounded_wait")
+
+
+def hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, grid: int,
+                   stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Read all of `buf` once (measurement of the read-only HBM ceiling); the
+    fold of what was read lands in `sink` (an int32 CUDA tensor)."""
+    if sink.dtype != torch.int32 or not sink.is_cuda:
+        raise ValueError("sink must be an int32 CUDA tensor")
+    _check(lib().pkv_hbm_read_probe(_dev(buf, "buf"), buf.numel() * buf.element_size(),
+                                    _dev(sink, "sink"), int(grid), _stream_handle(stream, buf.device)),
+           "pkv_hbm_read_probe")
 
 
 def kv_cache_write(key: torch.Tensor, value: torch.Tensor, slot_mapping: torch.Tensor,
