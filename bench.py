@@ -101,9 +101,11 @@ _SPLIT_CODE = [
 ]
 _CASCADE_CODE = [
     ("pkv_kernels.cuh", ["CascadeArgs", "load_slice", "lse_merge_cascade_kernel"]),
-    ("pkv_prefill.cuh", ["PrefillArgs", "PfShape", "PfBar", "tc_attend", "prefix_tc_kernel"]),
-    ("pagedkv.cu", ["make_query_map", "cascade_plan", "launch_prefix", "dispatch_prefix",
-                    "pkv_paged_attention_decode_cascade"]),
+    ("pkv_prefill.cuh", ["PrefillArgs", "PfShape", "PfBar", "TcMode", "tc_attend", "prefix_tc_kernel",
+                         "cascade_tc_kernel"]),
+    ("pagedkv.cu", ["make_query_map", "make_cache_map_4d", "cascade_plan", "launch_prefix",
+                    "dispatch_prefix", "launch_cascade_one_pass", "dispatch_cascade_one_pass",
+                    "cascade_one_pass", "pkv_paged_attention_decode_cascade"]),
 ]
 
 
@@ -454,13 +456,17 @@ class DecodeWorkload:
         ws_bytes = pkv.decode_workspace_bytes(B, Hq, Hkv, D, MB, bs, self.pt_req)
         self.launches_per_step = 2 + (1 if self.plan_np > 1 else 0)
         self.cas = None
+        self.one_pass = False
         if self.cascade:
             self.cas = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in
                         workloads.cascade_inputs(self.step, cfg.shared_prefix, cfg.samples).items()}
+            mpb, msb = self.cas["prefix_tables"].shape[1], self.cas["suffix_tables"].shape[1]
             ws_bytes = int(pkv.lib().pkv_decode_cascade_workspace_bytes(
-                B, Hq, Hkv, D, self.cas["prefix_tables"].shape[1], self.cas["suffix_tables"].shape[1],
-                self.cas["max_group_size"], bs, self.pt_req))
-            self.launches_per_step = 4
+                B, Hq, Hkv, D, mpb, msb, self.cas["max_group_size"], bs, self.pt_req))
+            self.one_pass, self.plan_np = pkv.decode_cascade_plan(
+                B, Hq, Hkv, D, mpb, msb, self.cas["max_group_size"],
+                self.cas["prefix_tables"].shape[0], bs, self.pt_req)
+            self.launches_per_step = 2 if self.one_pass else 4
         self.ws = torch.empty(max(16, ws_bytes), dtype=torch.uint8, device=dev)
         self.out = torch.empty_like(d["query"])
         self.flush = fits_in_l2(self.nbytes)
@@ -503,6 +509,8 @@ class DecodeWorkload:
         self.decode()
 
     def kernel_name(self) -> str:
+        if self.cascade and self.one_pass:
+            return "cascade_tc_kernel (one pass: prefix and own blocks)"
         if self.cascade:
             return "prefix_tc_kernel + paged_decode_kernel (suffixes) + lse_merge_cascade_kernel"
         return "paged_decode_kernel" + (" + lse_merge_kernel" if self.plan_np > 1 else "")
@@ -511,8 +519,10 @@ class DecodeWorkload:
         return committed_traffic(self.cfg.name, self.plan_np > 1 and not self.cascade, self.cascade)
 
     def method(self) -> dict:
-        return {"partition_tokens": self.plan_pt, "num_partitions": self.plan_np,
-                "cascade": self.cascade}
+        if self.cascade:
+            return {"cascade": "one pass" if self.one_pass else "split",
+                    "prefix_partitions": self.plan_np}
+        return {"partition_tokens": self.plan_pt, "num_partitions": self.plan_np, "cascade": False}
 
 
 def measure_decode_launches(w: DecodeWorkload, n: int, stream, flush_buf, sampler=None) -> dict:

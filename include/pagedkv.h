@@ -256,18 +256,36 @@ pkv_status pkv_paged_attention_prefill(const void *query, int num_tokens, const 
  *
  * Sequence b attends over prefix_tables[g] (prefix_lens[g] tokens) followed by
  * suffix_tables[b] (suffix_lens[b] tokens); sequences outside every group
- * attend over their suffix only.  Three kernels: the prefix pass (the
- * group's query rows, 128 per CTA, against each 64-key tile of the prefix on
- * the tcgen05 tensor cores, each prefix block read once per group), the
- * regular decode over the suffixes writing partial records, and a
- * log-sum-exp merge of both.
- * partition_tokens as for pkv_decode_plan (0: 512-token partitions).  Invalid
- * group bounds or prefix lengths set PKV_DEVFLAG_CONTEXT_RANGE.
+ * attend over their suffix only.  Two plans, both on the tcgen05 tensor
+ * cores for the group's query rows (128 per CTA):
+ *   one pass   one kernel: a CTA per (kv head, chunk of 128/G members) reads
+ *              its group's whole prefix once for all members' rows and then
+ *              each member's own blocks for that member's rows, and writes
+ *              the output; further CTAs take the sequences outside every
+ *              group.  The workspace is not used.
+ *   split      three kernels: the prefix in partitions (partial records per
+ *              row), the regular decode over the suffixes (partial records),
+ *              and a log-sum-exp merge of both.
+ * partition_tokens < 0 asks for the one pass; > 0 for the split plan with
+ * partitions of that many tokens (rounded up to a block multiple); 0 picks
+ * the one pass when num_groups > 0 and the groups' CTAs (num_groups x member
+ * chunks x num_kv_heads) number at least the SM count, else the split plan
+ * with 512-token partitions.  pkv_decode_cascade_plan tells which.  Invalid
+ * group bounds, prefix or suffix lengths set PKV_DEVFLAG_CONTEXT_RANGE.
+ * num_groups x member chunks above 65535 is PKV_ERR_UNSUPPORTED.
  */
 size_t pkv_decode_cascade_workspace_bytes(int batch, int num_heads, int num_kv_heads, int head_dim,
                                           int max_prefix_blocks, int max_suffix_blocks,
                                           int max_group_size, int block_size,
                                           int partition_tokens);
+/* The plan pkv_paged_attention_decode_cascade will use for these sizes:
+ * *one_pass = 1 for the one-pass kernel, else 0 and *prefix_partitions the
+ * prefix partitions of the split plan (either output may be NULL).  The
+ * workspace size above covers both plans. */
+pkv_status pkv_decode_cascade_plan(int batch, int num_heads, int num_kv_heads, int head_dim,
+                                   int max_prefix_blocks, int max_suffix_blocks, int max_group_size,
+                                   int num_groups, int block_size, int partition_tokens,
+                                   int *one_pass, int *prefix_partitions);
 pkv_status pkv_paged_attention_decode_cascade(
     const void *query, const void *key_cache, const void *value_cache,
     const int32_t *prefix_tables, int max_prefix_blocks, const int32_t *prefix_lens,

@@ -12,6 +12,7 @@ from .pagedkv import (  # noqa: F401
     BlockAllocator,
     PagedKVError,
     copy_blocks,
+    decode_cascade_plan,
     decode_plan,
     decode_workspace_bytes,
     device_flags,

@@ -90,6 +90,30 @@ pkv_status make_cache_map(CUtensorMap *map, const void *base, int64_t num_blocks
     return PKV_OK;
 }
 
+// The cache as a 4-D tensor {D, Hkv, bs, num_blocks}: a box is 64 columns x
+// 1 head x bs rows x 1 block.  Unlike the 3-D view, rows before a block's
+// first row are outside the tensor, so a load that starts at a negative row
+// reads zeros there (the one-pass cascade loads a partly filled block that
+// way, its valid rows at the end of the box).
+pkv_status make_cache_map_4d(CUtensorMap *map, const void *base, int64_t num_blocks, int bs,
+                             int Hkv, int D, pkv_dtype dt)
+{
+    EncodeTiledFn enc = encode_fn();
+    if (!enc)
+        return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable from the driver");
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)bs, (cuuint64_t)num_blocks};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)Hkv * D * 2, (cuuint64_t)bs * Hkv * D * 2};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)bs, 1};
+    cuuint32_t estride[4] = {1, 1, 1, 1};
+    CUresult r = enc(map, dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                     4, const_cast<void *>(base), dims, strides, box, estride,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS)
+        return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (4-D cache) failed (CUresult %d)", (int)r);
+    return PKV_OK;
+}
+
 // The query [T, Hq, D] seen as {D, Hq, T}; a box is 64 columns x the G heads
 // of one kv head x `tokens` query tokens: rows (token, head) of 128 bytes,
 // 128-byte swizzle, the prefill CTA's Q tile.  Rows past T read as zero.
@@ -581,6 +605,36 @@ cudaError_t dispatch_prefix(int D, int bs, const CUtensorMap &mq, const CUtensor
     return launch_prefix<128, 32, BF16>(mq, mk, mv, c, st);
 }
 
+// One-pass cascade: a CTA per (kv head, chunk of 128/G members of a group),
+// then free_chunks CTAs per kv head for the sequences outside every group.
+template <int D, int BS, bool BF16>
+cudaError_t launch_cascade_one_pass(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                                    const pkv::CascadeArgs &c, int free_chunks, cudaStream_t st)
+{
+    constexpr int smem = pkv::PfShape<D>::kSmemBytes;
+    auto kern = pkv::cascade_tc_kernel<D, BS, BF16>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)   // two CTAs (and their TMEM) per SM
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess)
+        return e;
+    const dim3 grid(1u, (unsigned)c.num_kv_heads,
+                    (unsigned)((size_t)c.num_groups * c.chunks + (size_t)free_chunks));
+    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, mk, mv, c);
+}
+
+template <bool BF16>
+cudaError_t dispatch_cascade_one_pass(int D, int bs, const CUtensorMap &mq, const CUtensorMap &mk,
+                                      const CUtensorMap &mv, const pkv::CascadeArgs &c,
+                                      int free_chunks, cudaStream_t st)
+{
+    if (D == 64 && bs == 16) return launch_cascade_one_pass<64, 16, BF16>(mq, mk, mv, c, free_chunks, st);
+    if (D == 64 && bs == 32) return launch_cascade_one_pass<64, 32, BF16>(mq, mk, mv, c, free_chunks, st);
+    if (D == 128 && bs == 16) return launch_cascade_one_pass<128, 16, BF16>(mq, mk, mv, c, free_chunks, st);
+    return launch_cascade_one_pass<128, 32, BF16>(mq, mk, mv, c, free_chunks, st);
+}
+
 }  // namespace
 
 extern "C" size_t pkv_decode_cascade_workspace_bytes(int batch, int num_heads, int num_kv_heads,
@@ -593,6 +647,44 @@ extern "C" size_t pkv_decode_cascade_workspace_bytes(int batch, int num_heads, i
                      max_group_size, block_size, partition_tokens, &c) != PKV_OK)
         return 0;
     return c.total;
+}
+
+namespace {
+
+// The one-pass choice of pkv_paged_attention_decode_cascade (see the header).
+bool cascade_one_pass(const CascadePlan &plan, int batch, int G, int num_kv_heads, int num_groups,
+                      int partition_tokens)
+{
+    const int per_cta = pkv::kPfRows / G;
+    const int64_t free_chunks = (batch + per_cta - 1) / per_cta;
+    const int64_t group_chunks = (int64_t)num_groups * plan.chunks;
+    return num_groups > 0 && group_chunks + free_chunks <= 65535 &&
+           (partition_tokens < 0 ||
+            (partition_tokens == 0 && group_chunks * num_kv_heads >= kPlanSmCount));
+}
+
+}  // namespace
+
+extern "C" pkv_status pkv_decode_cascade_plan(int batch, int num_heads, int num_kv_heads, int head_dim,
+                                              int max_prefix_blocks, int max_suffix_blocks,
+                                              int max_group_size, int num_groups, int block_size,
+                                              int partition_tokens, int *one_pass,
+                                              int *prefix_partitions)
+{
+    CascadePlan plan;
+    pkv_status s = cascade_plan(batch, num_heads, num_kv_heads, head_dim, max_prefix_blocks,
+                                max_suffix_blocks, max_group_size, block_size, partition_tokens, &plan);
+    if (s != PKV_OK)
+        return s;
+    if (num_groups < 0 || num_groups > batch)
+        return fail(PKV_ERR_INVALID_ARG, "num_groups %d (0 .. batch)", num_groups);
+    const bool op = cascade_one_pass(plan, batch, num_heads / num_kv_heads, num_kv_heads, num_groups,
+                                     partition_tokens);
+    if (one_pass)
+        *one_pass = op ? 1 : 0;
+    if (prefix_partitions)
+        *prefix_partitions = op ? 1 : plan.pp;
+    return PKV_OK;
 }
 
 extern "C" pkv_status pkv_paged_attention_decode_cascade(
@@ -639,8 +731,54 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const float scale_log2 = (float)((double)scale * 1.4426950408889634);
 
+    // One pass (prefix and own blocks in one CTA, no records, no merge) when
+    // asked for (partition_tokens < 0) or, automatically, when the groups'
+    // CTAs alone fill the GPU; else the prefix is split into partitions.
+    const int G = num_heads / num_kv_heads;
+    const int free_chunks = (batch + pkv::kPfRows / G - 1) / (pkv::kPfRows / G);
+    if ((int64_t)num_groups * plan.chunks > 65535)
+        return fail(PKV_ERR_UNSUPPORTED, "num_groups x member chunks (%lld) above 65535",
+                    (long long)num_groups * plan.chunks);
+    const bool one_pass = cascade_one_pass(plan, batch, G, num_kv_heads, num_groups, partition_tokens);
+    if (one_pass) {
+        CUtensorMap mq, mk4, mv4;
+        if ((s = make_query_map(&mq, query, batch, num_heads, head_dim, G, pkv::kPfRows / G, dtype)) != PKV_OK)
+            return s;
+        if ((s = make_cache_map_4d(&mk4, key_cache, num_blocks, block_size, num_kv_heads, head_dim,
+                                   dtype)) != PKV_OK)
+            return s;
+        if ((s = make_cache_map_4d(&mv4, value_cache, num_blocks, block_size, num_kv_heads, head_dim,
+                                   dtype)) != PKV_OK)
+            return s;
+        pkv::CascadeArgs c{};
+        c.query = static_cast<const uint16_t *>(query);
+        c.prefix_tables = prefix_tables;
+        c.prefix_lens = prefix_lens;
+        c.group_start = group_start;
+        c.batch = batch;
+        c.max_prefix_blocks = max_prefix_blocks;
+        c.num_groups = num_groups;
+        c.max_group_size = max_group_size;
+        c.num_heads = num_heads;
+        c.num_kv_heads = num_kv_heads;
+        c.group = G;
+        c.num_blocks = (int)num_blocks;
+        c.chunks = plan.chunks;
+        c.scale_log2 = scale_log2;
+        c.suffix_tables = suffix_tables;
+        c.suffix_lens = suffix_lens;
+        c.out = static_cast<uint16_t *>(out);
+        c.max_suffix_blocks = max_suffix_blocks;
+        cudaError_t e = dtype == PKV_BF16
+                            ? dispatch_cascade_one_pass<true>(head_dim, block_size, mq, mk4, mv4, c, free_chunks, st)
+                            : dispatch_cascade_one_pass<false>(head_dim, block_size, mq, mk4, mv4, c, free_chunks, st);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cascade_tc_kernel launch");
+        return PKV_OK;
+    }
+
     // level 1: shared prefixes, one pass per group
-    pkv::CascadeArgs c;
+    pkv::CascadeArgs c{};
     c.query = static_cast<const uint16_t *>(query);
     c.prefix_tables = prefix_tables;
     c.prefix_lens = prefix_lens;

@@ -555,7 +555,10 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // partition's record (max, normaliser, normalised row); level 2 (the decode
 // kernel over each sequence's own suffix, records only) and the cascade merge
 // below complete the result, which equals the decode over the concatenated
-// table.
+// table.  When there are enough groups to fill the GPU, one kernel does it all
+// instead (cascade_tc_kernel, pkv_prefill.cuh): a CTA per (kv head, chunk of
+// members) reads the group's whole prefix once and then each member's own
+// blocks, and writes the output rows; no records, no merge.
 struct CascadeArgs {
     const uint16_t *query;           // [B, Hq, D]
     const int32_t *prefix_tables;    // [num_groups, max_prefix_blocks]
@@ -576,6 +579,11 @@ struct CascadeArgs {
     int num_parts;                   // prefix partitions
     int chunks;                      // member chunks per group
     float scale_log2;
+    // one-pass cascade (prefix and every member's own blocks in one CTA)
+    const int32_t *suffix_tables;    // [batch, max_suffix_blocks]
+    const int32_t *suffix_lens;      // [batch]
+    uint16_t *out;                   // [B, Hq, D]
+    int max_suffix_blocks;
 };
 
 // Cascade merge: row (b, h) = its group's prefix records (partitions of the

@@ -1,8 +1,10 @@
 // pkv_prefill.cuh -- many query rows over the paged KV cache on the
 // 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory):
-// chunked prefill (prefill_tc_kernel) and the shared-prefix pass of cascade
+// chunked prefill (prefill_tc_kernel), the shared-prefix pass of cascade
 // decode (prefix_tc_kernel, which differs only in its work map, no causal
-// mask, and its output: partition records for the cascade merge).
+// mask, and its output: partition records for the cascade merge), and the
+// one-pass cascade decode (cascade_tc_kernel: a group's prefix and then each
+// member's own blocks, output rows).
 //
 // Sequence b brings C_b = query_start[b+1] - query_start[b] new tokens, the
 // last C_b of its L_b = context_lens[b] cached tokens (their K/V were written
@@ -116,11 +118,29 @@ enum PfBar {
 // refilled (S_{j+2}) only after P_j V_j has completed: no barrier can run two
 // phases ahead of its waiter.
 
-// The body shared by the chunked prefill (PREFIX = false: causal rows of one
-// sequence's chunk) and the prefix pass of cascade decode (PREFIX = true: the
-// query rows of a group's members over one partition of their shared prefix,
-// written as partition records for the merge).
-template <int D, int BS, bool BF16, bool PREFIX>
+// What a CTA of the shared body computes.
+enum TcMode : int {
+    // causal rows of one sequence's chunk; output rows
+    kTcPrefill = 0,
+    // the query rows of a group's members over one partition of their shared
+    // prefix; partition records for the cascade merge
+    kTcPrefix = 1,
+    // the query rows of a group's members over the group's whole prefix, then
+    // each member's rows over that member's own blocks (the other rows see
+    // none of them); output rows.  Extra CTAs at the end of the grid take the
+    // sequences outside every group (own blocks only).
+    kTcCascade = 2,
+};
+
+// One-pass cascade: the keys of a member's own blocks are taken in the order
+// (last block, block 0, block 1, ...), and the last block, when partly
+// filled, is loaded shifted so that its valid rows end the block's 16 or 32
+// rows (the rows before them lie outside the block and read as zero).  The
+// valid keys of every key tile are then one contiguous range of its columns.
+// Attention does not depend on the order of the keys.
+
+// The body shared by the three modes.
+template <int D, int BS, bool BF16, int MODE>
 __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
                                           const CUtensorMap *tm_v, const PrefillArgs &a,
                                           const CascadeArgs &c)
@@ -145,12 +165,13 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
     const int kvh = blockIdx.y;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int G = PREFIX ? c.group : a.group;
-    const int TT = kPfRows / G;   // query tokens (prefix: group members) per CTA
+    constexpr bool kCas = MODE != kTcPrefill;   // a cascade mode: c, not a
+    const int G = kCas ? c.group : a.group;
+    const int TT = kPfRows / G;   // query tokens (cascade: group members) per CTA
     const int R = TT * G;         // rows in use (128 when G divides 128)
-    const int num_heads = PREFIX ? c.num_heads : a.num_heads;
-    const int num_blocks = PREFIX ? c.num_blocks : a.num_blocks;
-    const float scale_log2 = PREFIX ? c.scale_log2 : a.scale_log2;
+    const int num_heads = kCas ? c.num_heads : a.num_heads;
+    const int num_blocks = kCas ? c.num_blocks : a.num_blocks;
+    const float scale_log2 = kCas ? c.scale_log2 : a.scale_log2;
 
     if (threadIdx.x == 0) {
         mbar_init(bar(kBarQFull), 1);
@@ -187,7 +208,15 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
     // all of them (prefix).
     int rows, row0, q_tok0, p_max, pos0, rec_part = 0;
     const int32_t *trow;
-    if constexpr (!PREFIX) {
+    // one-pass cascade: members first .. first + n_mem - 1 (the CTA's query
+    // rows, G per member); prefix of Lp tokens; lane l of every warp holds the
+    // key counts of members l, l + 32, l + 64, l + 96 (0 for a member another
+    // CTA covers); sequences outside every group are those before gs0 or
+    // from gsN on
+    int n_mem = 0, Lp = 0, gs0 = 0, gsN = 0, nt_cas = 0;
+    bool grouped = false;
+    int mlen[4] = {0, 0, 0, 0};
+    if constexpr (MODE == kTcPrefill) {
         const int tile = blockIdx.x;
         const int b = blockIdx.z;
         const int q0 = __ldg(a.query_start + b);
@@ -212,7 +241,7 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         pos0 = L - C + i0;                          // the first row's last key
         p_max = L - C + min(C, i0 + TT) - 1;        // last key any row of the CTA sees
         trow = a.block_tables + (size_t)b * a.max_blocks;
-    } else {
+    } else if constexpr (MODE == kTcPrefix) {
         const int pp = blockIdx.x;
         const int g = blockIdx.z / c.chunks;
         const int mc = blockIdx.z - g * c.chunks;
@@ -243,9 +272,118 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         pos0 = p_max;
         trow = c.prefix_tables + (size_t)g * c.max_prefix_blocks + tok0 / BS;
         rec_part = pp;
+    } else {
+        const int gz = c.num_groups * c.chunks;
+        int first;
+        const int z = blockIdx.z;
+        if (c.num_groups > 0) {
+            gs0 = min(max(__ldg(c.group_start), 0), c.batch);
+            gsN = min(max(__ldg(c.group_start + c.num_groups), gs0), c.batch);
+        }
+        if (z < gz) {
+            const int g = z / c.chunks;
+            const int mc = z - g * c.chunks;
+            first = __ldg(c.group_start + g);
+            int count = __ldg(c.group_start + g + 1) - first;
+            if (first < 0 || count < 0 || first + count > c.batch || count > c.max_group_size) {
+                if (threadIdx.x == 0 && kvh == 0 && mc == 0)
+                    raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+                first = first < 0 ? 0 : (first > c.batch ? c.batch : first);
+                count = count < 0 ? 0 : count;
+                count = min(count, min(c.max_group_size, c.batch - first));
+            }
+            Lp = __ldg(c.prefix_lens + g);
+            const int span = c.max_prefix_blocks * BS;
+            if (Lp < 0 || Lp > span || Lp % BS != 0) {
+                if (threadIdx.x == 0 && kvh == 0 && mc == 0)
+                    raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+                Lp = Lp < 0 ? 0 : (Lp > span ? span : Lp - Lp % BS);
+            }
+            first += mc * TT;
+            n_mem = min(TT, count - mc * TT);
+            trow = c.prefix_tables + (size_t)g * c.max_prefix_blocks;
+            grouped = true;
+        } else {
+            first = (z - gz) * TT;
+            n_mem = min(TT, c.batch - first);
+            trow = c.prefix_tables;                 // not read: Lp = 0
+            if (n_mem > 0 && first >= gs0 && first + n_mem <= gsN)
+                n_mem = 0;                          // every sequence here is in a group
+        }
+        if (n_mem <= 0)
+            return;                                 // whole CTA, before TMEM is touched
+        const int sspan = c.max_suffix_blocks * BS;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int m = lane + 32 * i;
+            if (m < n_mem) {
+                const int b = first + m;
+                if (grouped || b < gs0 || b >= gsN) {
+                    int Ls = __ldg(c.suffix_lens + b);
+                    if (Ls < 0 || Ls > sspan) {
+                        raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+                        Ls = Ls < 0 ? 0 : sspan;
+                    }
+                    mlen[i] = Ls;
+                }
+            }
+        }
+        int tiles = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            tiles += (mlen[i] + kPfKeys - 1) / kPfKeys;
+        nt_cas = (Lp + kPfKeys - 1) / kPfKeys + __reduce_add_sync(0xffffffffu, tiles);
+        rows = n_mem * G;
+        row0 = 0;
+        q_tok0 = first;
+        pos0 = p_max = 0;                           // unused: the walk gives each tile's keys
+        if (nt_cas == 0) {
+            // no keys for any row: zero output rows (the rows this CTA owns)
+            for (int idx = threadIdx.x; idx < rows * D; idx += kPfThreads) {
+                const int r = idx / D;
+                const int b = first + r / G;
+                if (grouped || b < gs0 || b >= gsN)
+                    c.out[((size_t)b * num_heads + (size_t)kvh * G + r % G) * D + idx % D] = 0;
+            }
+            return;
+        }
     }
-    const int nt = p_max / kPfKeys + 1;             // key tiles
-    const int nblk = p_max / BS + 1;                // cache blocks read
+    // key count of member m (warp-uniform m), from the lanes' registers
+    auto member_len = [&](int m) -> int {
+        const int v = m < 32 ? mlen[0] : (m < 64 ? mlen[1] : (m < 96 ? mlen[2] : mlen[3]));
+        return __shfl_sync(0xffffffffu, v, m & 31);
+    };
+    // the next member after m with keys (n_mem if none)
+    auto next_member = [&](int m) -> int {
+        for (++m; m < n_mem; ++m)
+            if (member_len(m) > 0)
+                break;
+        return m;
+    };
+    // one-pass cascade: the key tiles in order -- segment m = -1 is the
+    // prefix, m >= 0 member m's own blocks; tile k of the segment, whose
+    // keys number len
+    struct Walk {
+        int m, k, len;
+    };
+    auto walk_start = [&]() -> Walk {
+        Walk w{-1, 0, Lp};
+        if (w.len == 0) {
+            w.m = next_member(-1);
+            w.len = w.m < n_mem ? member_len(w.m) : 0;
+        }
+        return w;
+    };
+    auto walk_next = [&](Walk &w) -> bool {         // true: a new segment starts
+        if (++w.k * kPfKeys < w.len)
+            return false;
+        w.m = next_member(w.m);
+        w.len = w.m < n_mem ? member_len(w.m) : 0;
+        w.k = 0;
+        return true;
+    };
+    const int nt = MODE == kTcCascade ? nt_cas : p_max / kPfKeys + 1;   // key tiles
+    const int nblk = p_max / BS + 1;                // cache blocks read (other modes)
 
     // ---- tensor memory ----
     if (warp == 5) {
@@ -274,9 +412,9 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         {
             // the whole warp walks the tiles: block ids are read 32 at a time,
             // one per lane, and lane 0 issues the copies
-            // prefill: the sequence's other CTAs reread these blocks; prefix:
+            // prefill: the sequence's other CTAs reread these blocks; cascade:
             // each is read once per group and kv head
-            const uint64_t policy = PREFIX ? policy_evict_first() : policy_evict_normal();
+            const uint64_t policy = kCas ? policy_evict_first() : policy_evict_normal();
             if (is_k && lane == 0) {
                 mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(Sh::kHalves * R * 128));
 #pragma unroll
@@ -284,6 +422,81 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                     tma_load_3d(sQ + h * Sh::kQHalf, tm_q, bar(kBarQFull), h * 64, kvh * G, q_tok0,
                                 policy);
             }
+            if constexpr (MODE == kTcCascade) {
+                if (!is_k) {
+                    // keys outside a tile's valid columns meet these V rows with
+                    // weight 0, so they must be finite: the ring starts at zero
+                    // and then only holds loaded rows or rows read as zero
+                    uint4 *vr = reinterpret_cast<uint4 *>(data + Sh::kVOff);
+                    for (int i = lane; i < kPfVStages * Sh::kKVBytes / 16; i += 32)
+                        vr[i] = make_uint4(0u, 0u, 0u, 0u);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                // block ids of window w of a segment, lane l: entry w + l of the
+                // segment's block order (the prefix in table order; a member's
+                // last block first, then its blocks from 0)
+                auto load_ids = [&](const Walk &g, int w) -> int {
+                    const int nb = (g.len + BS - 1) / BS;
+                    const int r = w + lane;
+                    if (g.m >= n_mem || r >= nb)
+                        return 0;
+                    if (g.m < 0)
+                        return __ldg(trow + r);
+                    const int32_t *t = c.suffix_tables + (size_t)(q_tok0 + g.m) * c.max_suffix_blocks;
+                    return __ldg(t + (r == 0 ? nb - 1 : r - 1));
+                };
+                Walk wk = walk_start();
+                int ids = load_ids(wk, 0);
+                // the next segment's first ids are read one segment ahead
+                Walk nx = wk;
+                nx.k = (nx.len + kPfKeys - 1) / kPfKeys - 1;
+                walk_next(nx);
+                int ids_next = load_ids(nx, 0);
+                for (int j = 0; j < nt; ++j) {
+                    const int s = j % NS;
+                    if (j >= NS) {
+                        const bool free_ = mbar_wait_bounded(bar(empty0 + s), (uint32_t)((j / NS - 1) & 1),
+                                                             kWaitLimitNs);
+                        if (!__all_sync(0xffffffffu, free_)) {
+                            if (lane == 0)
+                                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+                            break;
+                        }
+                    }
+                    const int nb_seg = (wk.len + BS - 1) / BS;
+                    const int kb0 = wk.k * BPT;            // a tile never straddles 32 ids
+                    const int nb = min(BPT, nb_seg - kb0);
+                    if (kb0 > 0 && (kb0 & 31) == 0)
+                        ids = load_ids(wk, kb0);
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(bar(full0 + s), (uint32_t)(nb * BS * D * 2));
+                    __syncwarp();
+                    const int i = lane / Sh::kHalves;
+                    const int h = lane - i * Sh::kHalves;
+                    int blk = __shfl_sync(0xffffffffu, ids, (kb0 + min(i, BPT - 1)) & 31);
+                    if (i < nb) {
+                        if ((unsigned)blk >= (unsigned)num_blocks) {
+                            if (h == 0)
+                                raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
+                            blk = 0;
+                        }
+                        // a member's partly filled last block is shifted to end at
+                        // its slot's last row; the rows before it read as zero
+                        const int shift = (wk.m >= 0 && kb0 + i == 0) ? wk.len - nb_seg * BS : 0;
+                        tma_load_4d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
+                                    bar(full0 + s), h * 64, kvh, shift, blk, policy);
+                    }
+                    issued = j + 1;
+                    if (walk_next(wk)) {
+                        ids = ids_next;
+                        nx = wk;
+                        nx.k = (nx.len + kPfKeys - 1) / kPfKeys - 1;
+                        walk_next(nx);
+                        ids_next = load_ids(nx, 0);
+                    }
+                }
+            } else {
             int ids = 0;
             for (int j = 0; j < nt; ++j) {
                 const int s = j % NS;
@@ -319,8 +532,9 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 }
                 issued = j + 1;
             }
+            }
         }
-        if (!is_k && issued == nt) {
+        if (MODE != kTcCascade && !is_k && issued == nt) {
             // V rows of the last tile past p_max (the context's tail in its last
             // block, and blocks never loaded) are cleared once the tile landed
             const int j = nt - 1;
@@ -397,7 +611,8 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 ok = mbar_wait_bounded(bar(kBarPFull + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
                      mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((j / kPfVStages) & 1),
                                        kWaitLimitNs) &&
-                     (j + 1 < nt || mbar_wait_bounded(bar(kBarVTail), 0u, kWaitLimitNs));
+                     (MODE == kTcCascade || j + 1 < nt ||
+                      mbar_wait_bounded(bar(kBarVTail), 0u, kWaitLimitNs));
                 if (!ok)
                     break;
                 tc_fence_after();
@@ -425,7 +640,7 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
         const int grow = row0 + r;                  // row within the sequence
         const bool real = r < R && grow < rows;
-        const int pos = real && !PREFIX ? pos0 + r / G : p_max;
+        const int pos = real && MODE == kTcPrefill ? pos0 + r / G : p_max;
         float m_used = kNegInf;
         float l = 0.f;
         bool ok = true;
@@ -435,6 +650,7 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         const bool fold = sc > 0.f;
         const float sm = fold ? 1.f : sc;       // applied before the maximum
         const float se = fold ? sc : 1.f;       // applied in the exponent
+        Walk sw = walk_start();                     // one-pass cascade: the tile walk
         for (int j = 0; j < nt; ++j) {
             const int s = j & 1;
             ok = mbar_wait_bounded(bar(kBarSFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
@@ -443,6 +659,27 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 break;
             }
             tc_fence_after();
+            // one-pass cascade: the tile's valid key columns [clo, chi) and the
+            // query rows [rlo, rhi) that see them (the prefix: every row; a
+            // member's own blocks: that member's G rows)
+            int clo = 0, chi = kPfKeys, rlo = 0, rhi = rows;
+            if constexpr (MODE == kTcCascade) {
+                const int nbs = (sw.len + BS - 1) / BS;
+                if (sw.m < 0) {
+                    chi = min(kPfKeys, sw.len - sw.k * kPfKeys);
+                } else {
+                    clo = sw.k == 0 ? nbs * BS - sw.len : 0;
+                    chi = BS * min(BPT, nbs - sw.k * BPT);
+                    rlo = sw.m * G;
+                    rhi = rlo + G;
+                }
+            }
+            // no row of this warp sees the tile: its weights are all zero
+            const bool warp_off = MODE == kTcCascade && (rhi <= warp * 32 || rlo >= warp * 32 + 32);
+            uint32_t pk[32];
+            bool resc = false;
+            float alpha = 1.f;
+            if (!warp_off) {
             uint32_t raw[64];
             tmem_ld64(tmem + lane_base + s * kPfKeys, raw);
             // eight independent max / sum chains, not 64-long ones
@@ -452,7 +689,13 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             for (int i = 0; i < 8; ++i)
                 mx[i] = kNegInf;
             const int t0 = j * kPfKeys;
-            if (t0 + kPfKeys - 1 <= pos0) {         // every key visible to every row
+            bool all_visible;
+            if constexpr (MODE == kTcCascade)
+                all_visible = clo == 0 && chi == kPfKeys && rlo <= warp * 32 && rhi >= warp * 32 + 32;
+            else
+                all_visible = t0 + kPfKeys - 1 <= pos0;
+            const bool row_on = r >= rlo && r < rhi;
+            if (all_visible) {                      // every key visible to every row
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     x[c] = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
@@ -462,19 +705,23 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const float v = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
-                    x[c] = t0 + c <= pos ? v : kNegInf;
+                    bool vis;
+                    if constexpr (MODE == kTcCascade)
+                        vis = row_on && c >= clo && c < chi;
+                    else
+                        vis = t0 + c <= pos;
+                    x[c] = vis ? v : kNegInf;
                     mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
             }
             const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * se;
-            const bool resc = mt > m_used + 8.f;    // first tile: m_used = -inf
+            resc = mt > m_used + 8.f;               // first tile: m_used = -inf
             const float m_new = resc ? mt : m_used;
-            const float alpha = resc ? ex2(m_used - m_new) : 1.f;
+            alpha = resc ? ex2(m_used - m_new) : 1.f;
             const float msub = m_new == kNegInf ? 0.f : m_new;
             // the row sum is taken over the rounded weights the MMA multiplies,
             // so the normalised weights sum to one exactly
-            uint32_t pk[32];
             float rsv[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -488,6 +735,11 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
             l = l * alpha + rs;
             m_used = m_new;
+            } else {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                    pk[c] = 0u;
+            }
             if (j > 0) {
                 // Wait for P_{j-1} V_{j-1}: O then holds it (for the rescale),
                 // and O_DONE stays within one phase of this warp, so the
@@ -520,6 +772,8 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar(kBarPFull + s));
+            if constexpr (MODE == kTcCascade)
+                walk_next(sw);
         }
         if (ok)
             ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((nt - 1) & 1), kWaitLimitNs);
@@ -528,13 +782,19 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             const float inv = l > 0.f ? 1.f / l : 0.f;
             // query row (q_tok0 + r / G, head kvh * G + r % G): row0 is a multiple of G
             const size_t orow_i = (size_t)(q_tok0 + r / G) * num_heads + (size_t)kvh * G + r % G;
-            if constexpr (!PREFIX) {
-                uint4 *orow = reinterpret_cast<uint4 *>(a.out + orow_i * D);
+            if constexpr (MODE != kTcPrefix) {
+                // one-pass cascade: only the rows of sequences this CTA covers
+                bool own = real;
+                if constexpr (MODE == kTcCascade) {
+                    const int b = q_tok0 + r / G;
+                    own = real && (grouped || b < gs0 || b >= gsN);
+                }
+                uint4 *orow = reinterpret_cast<uint4 *>((MODE == kTcPrefill ? a.out : c.out) + orow_i * D);
 #pragma unroll 1
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tO + lane_base + c0, o);
-                    if (real) {
+                    if (own) {
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             uint32_t w[4];
@@ -588,7 +848,7 @@ __global__ void __launch_bounds__(kPfThreads, 2)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a)
 {
-    tc_attend<D, BS, BF16, false>(&tm_q, &tm_k, &tm_v, a, CascadeArgs{});
+    tc_attend<D, BS, BF16, kTcPrefill>(&tm_q, &tm_k, &tm_v, a, CascadeArgs{});
 }
 
 template <int D, int BS, bool BF16>
@@ -596,7 +856,18 @@ __global__ void __launch_bounds__(kPfThreads, 2)
 prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const CascadeArgs c)
 {
-    tc_attend<D, BS, BF16, true>(&tm_q, &tm_k, &tm_v, PrefillArgs{}, c);
+    tc_attend<D, BS, BF16, kTcPrefix>(&tm_q, &tm_k, &tm_v, PrefillArgs{}, c);
+}
+
+// One-pass cascade decode: tm_k / tm_v view the caches as 4-D tensors
+// {head_dim, num_kv_heads, block_size, num_blocks} (box 64 x 1 x block_size
+// x 1), so that a shifted load of a partly filled block reads zeros before it.
+template <int D, int BS, bool BF16>
+__global__ void __launch_bounds__(kPfThreads, 2)
+cascade_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v, const CascadeArgs c)
+{
+    tc_attend<D, BS, BF16, kTcCascade>(&tm_q, &tm_k, &tm_v, PrefillArgs{}, c);
 }
 
 }  // namespace pkv

@@ -74,6 +74,8 @@ def lib() -> ctypes.CDLL:
                                                   i32, i32, i64, f32, P, i32, P]
         L.pkv_decode_cascade_workspace_bytes.restype = sz
         L.pkv_decode_cascade_workspace_bytes.argtypes = [i32] * 9
+        L.pkv_decode_cascade_plan.restype = i32
+        L.pkv_decode_cascade_plan.argtypes = [i32] * 10 + [pint, pint]
         L.pkv_paged_attention_decode_cascade.restype = i32
         L.pkv_paged_attention_decode_cascade.argtypes = [
             P, P, P, P, i32, P, P, i32, i32, P, i32, P, i32, i32, i32, i32, i32, i64, f32, i32, P,
@@ -310,6 +312,18 @@ def paged_attention_prefill(query: torch.Tensor, query_start: torch.Tensor, max_
         B, Hq, Hkv, D, bs, NB, float(scale), _dev(out, "out"), dt, _stream_handle(stream, query.device))
     _check(st, "pkv_paged_attention_prefill")
     return out
+
+
+def decode_cascade_plan(batch: int, num_heads: int, num_kv_heads: int, head_dim: int,
+                        max_prefix_blocks: int, max_suffix_blocks: int, max_group_size: int,
+                        num_groups: int, block_size: int, partition_tokens: int = 0) -> tuple:
+    """(one_pass, prefix_partitions) the cascade decode will use."""
+    op, pp = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().pkv_decode_cascade_plan(batch, num_heads, num_kv_heads, head_dim, max_prefix_blocks,
+                                         max_suffix_blocks, max_group_size, num_groups, block_size,
+                                         partition_tokens, ctypes.byref(op), ctypes.byref(pp)),
+           "pkv_decode_cascade_plan")
+    return bool(op.value), pp.value
 
 
 def paged_attention_decode_cascade(query: torch.Tensor, key_cache: torch.Tensor,

@@ -186,3 +186,14 @@ def test_hbm_read_probe_host_validation():
     assert L.pkv_hbm_read_probe(a16, 16, a16, 0, None) == pagedkv.ERR_INVALID_ARG   # empty grid
     assert L.pkv_hbm_read_probe(a16 + 8, 16, a16, 1, None) == pagedkv.ERR_MISALIGNED
     assert L.pkv_hbm_read_probe(a16, 16, a16 + 2, 1, None) == pagedkv.ERR_MISALIGNED
+
+
+def test_cascade_plan_choice():
+    # 32 groups x 8 kv heads fill the GPU: one pass; 12 x 8 do not: split in 512-token partitions
+    assert pkv.decode_cascade_plan(256, 32, 8, 128, 125, 16, 8, 32, 16, 0) == (True, 1)
+    assert pkv.decode_cascade_plan(96, 32, 8, 128, 125, 16, 8, 12, 16, 0) == (False, 4)
+    assert pkv.decode_cascade_plan(96, 32, 8, 128, 125, 16, 8, 12, 16, -1) == (True, 1)
+    assert pkv.decode_cascade_plan(96, 32, 8, 128, 125, 16, 8, 12, 16, 64) == (False, 32)
+    assert pkv.decode_cascade_plan(96, 32, 8, 128, 125, 16, 8, 0, 16, -1) == (False, 4)   # no groups
+    with pytest.raises(pkv.PagedKVError):
+        pkv.decode_cascade_plan(96, 32, 8, 128, 125, 16, 8, 97, 16, 0)                     # > batch

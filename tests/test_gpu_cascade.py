@@ -3,7 +3,12 @@
 The cascade computes exactly the decode over each sequence's full table
 (group prefix followed by its own blocks): the oracle runs the plain
 definition on the concatenated tables ("23.1 vLLM：高吞吐推理框架原理与部署",
-section 二.3: parallel samples share the prompt's blocks)."""
+section 二.3: parallel samples share the prompt's blocks).
+
+Both plans are covered: the split plan (prefix partitions as records, the
+suffix decode, a merge; partition_tokens > 0) and the one pass (a CTA per
+group chunk reads the prefix and then each member's own blocks;
+partition_tokens < 0); partition_tokens = 0 picks by size."""
 import numpy as np
 import pytest
 import torch
@@ -18,11 +23,14 @@ pytestmark = pytest.mark.gpu
 _DT = {"f16": torch.float16, "bf16": torch.bfloat16}
 
 
-def _cascade_case(groups, prefix_blocks, suffix_tokens, Hq, Hkv, D, bs, dtype, seed):
+def _cascade_case(groups, prefix_blocks, suffix_tokens, Hq, Hkv, D, bs, dtype, seed, before=0,
+                  after=0):
     """groups: sizes of consecutive groups (0-prefix groups allowed);
-    prefix_blocks[g]: shared blocks; suffix_tokens[b]: own tokens."""
+    prefix_blocks[g]: shared blocks; suffix_tokens[b]: own tokens;
+    `before` / `after` sequences outside every group (own tokens only)."""
     g = torch.Generator().manual_seed(seed)
-    B = sum(groups)
+    B = before + sum(groups) + after
+    assert len(suffix_tokens) == B
     sfx_blocks = [-(-t // bs) for t in suffix_tokens]
     need = sum(prefix_blocks) + sum(sfx_blocks)
     NB = need + 7
@@ -37,17 +45,20 @@ def _cascade_case(groups, prefix_blocks, suffix_tokens, Hq, Hkv, D, bs, dtype, s
     for b, n in enumerate(sfx_blocks):
         suffix_tables[b, :n] = torch.tensor(perm[cur:cur + n], dtype=torch.int32)
         cur += n
-    group_start = torch.tensor(np.concatenate([[0], np.cumsum(groups)]), dtype=torch.int32)
+    group_start = torch.tensor(before + np.concatenate([[0], np.cumsum(groups)]), dtype=torch.int32)
     prefix_lens = torch.tensor([n * bs for n in prefix_blocks], dtype=torch.int32)
     suffix_lens = torch.tensor(suffix_tokens, dtype=torch.int32)
     # full tables for the oracle: prefix blocks, then own blocks
     full_lens, rows = [], []
+    owner = [None] * B
     for gi, size in enumerate(groups):
         for m in range(size):
-            b = int(group_start[gi]) + m
-            row = prefix_tables[gi, :prefix_blocks[gi]].tolist() + suffix_tables[b, :sfx_blocks[b]].tolist()
-            rows.append(row)
-            full_lens.append(prefix_blocks[gi] * bs + suffix_tokens[b])
+            owner[int(group_start[gi]) + m] = gi
+    for b in range(B):
+        gi = owner[b]
+        pre = prefix_tables[gi, :prefix_blocks[gi]].tolist() if gi is not None else []
+        rows.append(pre + suffix_tables[b, :sfx_blocks[b]].tolist())
+        full_lens.append((prefix_blocks[gi] * bs if gi is not None else 0) + suffix_tokens[b])
     mb = max(1, max(len(r) for r in rows))
     full = torch.full((B, mb), -1, dtype=torch.int32)
     for b, r in enumerate(rows):
@@ -112,7 +123,7 @@ def test_cascade_irregular_groups(D, bs, dtype):
     suffix_tokens = [7, 0, 33, 100, 1, 16, 0]
     case = _cascade_case(groups, prefix_blocks, suffix_tokens, 8, 2, D, bs, dtype, seed=D + bs)
     ref = _oracle(case)
-    for pt in (0, 64):
+    for pt in (0, 64, -1):                  # auto (split here), split, one pass
         err, idx, finite = max_abs_err(_run(case, pt), ref)
         assert finite and err <= TOL[dtype], (pt, err, idx)
 
@@ -126,5 +137,54 @@ def test_cascade_group_shapes(G, size):
     case = _cascade_case(groups, [12, 20], list(range(1, 2 * size + 1)), G * Hkv, Hkv, 128, 16,
                          "bf16", seed=G * 100 + size)
     ref = _oracle(case)
-    err, idx, finite = max_abs_err(_run(case), ref)
-    assert finite and err <= TOL["bf16"], (err, idx)
+    for pt in (0, -1):
+        err, idx, finite = max_abs_err(_run(case, pt), ref)
+        assert finite and err <= TOL["bf16"], (pt, err, idx)
+
+
+@pytest.mark.parametrize("D,bs,dtype", [(128, 16, "bf16"), (64, 32, "f16"), (128, 32, "f16"),
+                                        (64, 16, "bf16")])
+def test_cascade_sequences_outside_groups(D, bs, dtype):
+    """Sequences before and after the groups attend over their own blocks only."""
+    groups = [4, 2]
+    before, after = 3, 5
+    B = before + sum(groups) + after
+    suffix = [1, 0, 40, 17, 16, 15, 64, 65, 0, 3, 100, 33, 2, 129][:B]
+    case = _cascade_case(groups, [6, 3], suffix, 8, 2, D, bs, dtype, seed=D * 3 + bs, before=before,
+                         after=after)
+    ref = _oracle(case)
+    for pt in (64, -1):
+        err, idx, finite = max_abs_err(_run(case, pt), ref)
+        assert finite and err <= TOL[dtype], (pt, err, idx)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_cascade_one_pass_long_and_edge_suffixes(bs):
+    """Own-block lengths around block and tile edges, and own blocks beyond one
+    32-entry window of block ids (more than 512 tokens at 16 per block)."""
+    suffix = [0, 1, bs - 1, bs, bs + 1, 63, 64, 65, 127, 128, 129, 700, 1100, 2, 0, 513]
+    groups = [8, 8]
+    case = _cascade_case(groups, [9, 1], suffix, 16, 4, 128, bs, "bf16", seed=bs + 5)
+    ref = _oracle(case)
+    for pt in (0, -1, 128):
+        err, idx, finite = max_abs_err(_run(case, pt), ref)
+        assert finite and err <= TOL["bf16"], (pt, err, idx)
+
+
+def test_cascade_one_pass_garbage_past_the_end():
+    """Cells past each sequence's last token (in its last block) hold NaN: they
+    are never weighted, so the output stays finite and within tolerance."""
+    groups = [5, 3]
+    suffix = [3, 17, 30, 1, 9, 40, 2, 33]
+    case = _cascade_case(groups, [4, 2], suffix, 16, 4, 128, 16, "bf16", seed=91)
+    ref = _oracle(case)
+    bs = 16
+    for b, n in enumerate(suffix):
+        nb = -(-n // bs)
+        if n % bs:
+            blk = int(case["suffix_tables"][b, nb - 1])
+            case["key_cache"][blk, n % bs:] = float("nan")
+            case["value_cache"][blk, n % bs:] = float("nan")
+    for pt in (64, -1):
+        err, idx, finite = max_abs_err(_run(case, pt), ref)
+        assert finite and err <= TOL["bf16"], (pt, err, idx)

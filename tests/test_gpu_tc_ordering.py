@@ -16,9 +16,9 @@ with the device flag word clear afterwards (no bounded wait expired).
 The prefill case is the shape that exposed an ordering fault before: chunks
 of 7 tokens over 520 cached keys, group size 4, bf16 (9 key tiles, so the
 last P V phases are still open when the softmax warps finish).  The cascade
-case is the shared-prefix workload's shape at reduced batch: groups of 8
+cases are the shared-prefix workload's shape at reduced batch: groups of 8
 samples sharing a 2000-token prefix ("23.1 vLLM：高吞吐推理框架原理与部署",
-section 二.3).
+section 二.3), through the split plan and through the one pass.
 """
 import numpy as np
 import pytest
@@ -68,7 +68,8 @@ def test_prefill_short_chunks_over_long_context_repeated():
     assert not bad, f"{len(bad)} of {PREFILL_RUNS} runs differ from the first: {bad[:10]}"
 
 
-def test_cascade_prefix_pass_repeated():
+@pytest.mark.parametrize("partition_tokens", [512, -1])   # prefix pass + merge; one pass
+def test_cascade_repeated(partition_tokens):
     groups = [8] * 12                        # 96 sequences, 12 prompts x 8 samples
     rng = np.random.default_rng(7)
     suffix = [int(x) for x in rng.integers(1, 257, size=sum(groups))]
@@ -78,7 +79,8 @@ def test_cascade_prefix_pass_repeated():
     runs = [pkv.paged_attention_decode_cascade(
         d["query"], d["key_cache"], d["value_cache"], d["prefix_tables"], d["prefix_lens"],
         d["group_start"], d["suffix_tables"], d["suffix_lens"], d["scale"],
-        max_group_size=d["max_group_size"]) for _ in range(CASCADE_RUNS)]
+        max_group_size=d["max_group_size"], partition_tokens=partition_tokens)
+        for _ in range(CASCADE_RUNS)]
     torch.cuda.synchronize()
     err, idx, finite = max_abs_err(runs[0], ref)
     assert finite and err <= TOL["bf16"], (err, idx)
