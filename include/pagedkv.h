@@ -258,7 +258,7 @@ pkv_status pkv_paged_attention_prefill(const void *query, int num_tokens, const 
  * suffix_tables[b] (suffix_lens[b] tokens); sequences outside every group
  * attend over their suffix only.  Two plans, both on the tcgen05 tensor
  * cores for the group's query rows (128 per CTA):
- *   one pass   one kernel: a CTA per (kv head, chunk of 128/G members) reads
+ *   one pass   one kernel: a CTA per (kv head, chunk of 32/G members) reads
  *              its group's whole prefix once for all members' rows and then
  *              each member's own blocks for that member's rows, and writes
  *              the output; further CTAs take the sequences outside every
@@ -268,8 +268,8 @@ pkv_status pkv_paged_attention_prefill(const void *query, int num_tokens, const 
  *              and a log-sum-exp merge of both.
  * partition_tokens < 0 asks for the one pass; > 0 for the split plan with
  * partitions of that many tokens (rounded up to a block multiple); 0 picks
- * the one pass when num_groups > 0 and the groups' CTAs (num_groups x member
- * chunks x num_kv_heads) number at least the SM count, else the split plan
+ * the one pass when num_groups > 0 and its CTAs (num_groups x chunks of 32/G
+ * members x num_kv_heads) number at least the SM count, else the split plan
  * with 512-token partitions.  pkv_decode_cascade_plan tells which.  Invalid
  * group bounds, prefix or suffix lengths set PKV_DEVFLAG_CONTEXT_RANGE.
  * num_groups x member chunks above 65535 is PKV_ERR_UNSUPPORTED.

@@ -605,7 +605,7 @@ cudaError_t dispatch_prefix(int D, int bs, const CUtensorMap &mq, const CUtensor
     return launch_prefix<128, 32, BF16>(mq, mk, mv, c, st);
 }
 
-// One-pass cascade: a CTA per (kv head, chunk of 128/G members of a group),
+// One-pass cascade: a CTA per (kv head, chunk of 32/G members of a group),
 // then free_chunks CTAs per kv head for the sequences outside every group.
 template <int D, int BS, bool BF16>
 cudaError_t launch_cascade_one_pass(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
@@ -651,16 +651,32 @@ extern "C" size_t pkv_decode_cascade_workspace_bytes(int batch, int num_heads, i
 
 namespace {
 
+// The one pass takes 32 query rows per CTA (32/G members): chunks of a group
+// and CTAs for the sequences outside every group, per kv head.
+constexpr int kOnePassRows = pkv::kCasRows;
+struct OnePassGrid {
+    int64_t group_chunks;   // member chunks of all groups
+    int chunks;             // member chunks per group
+    int free_chunks;        // chunks over the whole batch for ungrouped sequences
+};
+OnePassGrid one_pass_grid(int batch, int G, int max_group_size, int num_groups)
+{
+    const int per_cta = kOnePassRows / G;
+    OnePassGrid g;
+    g.chunks = (max_group_size + per_cta - 1) / per_cta;
+    g.group_chunks = (int64_t)num_groups * g.chunks;
+    g.free_chunks = (batch + per_cta - 1) / per_cta;
+    return g;
+}
+
 // The one-pass choice of pkv_paged_attention_decode_cascade (see the header).
-bool cascade_one_pass(const CascadePlan &plan, int batch, int G, int num_kv_heads, int num_groups,
+bool cascade_one_pass(int batch, int G, int num_kv_heads, int max_group_size, int num_groups,
                       int partition_tokens)
 {
-    const int per_cta = pkv::kPfRows / G;
-    const int64_t free_chunks = (batch + per_cta - 1) / per_cta;
-    const int64_t group_chunks = (int64_t)num_groups * plan.chunks;
-    return num_groups > 0 && group_chunks + free_chunks <= 65535 &&
+    const OnePassGrid g = one_pass_grid(batch, G, max_group_size, num_groups);
+    return num_groups > 0 && g.group_chunks + g.free_chunks <= 65535 &&
            (partition_tokens < 0 ||
-            (partition_tokens == 0 && group_chunks * num_kv_heads >= kPlanSmCount));
+            (partition_tokens == 0 && g.group_chunks * num_kv_heads >= kPlanSmCount));
 }
 
 }  // namespace
@@ -678,8 +694,8 @@ extern "C" pkv_status pkv_decode_cascade_plan(int batch, int num_heads, int num_
         return s;
     if (num_groups < 0 || num_groups > batch)
         return fail(PKV_ERR_INVALID_ARG, "num_groups %d (0 .. batch)", num_groups);
-    const bool op = cascade_one_pass(plan, batch, num_heads / num_kv_heads, num_kv_heads, num_groups,
-                                     partition_tokens);
+    const bool op = cascade_one_pass(batch, num_heads / num_kv_heads, num_kv_heads, max_group_size,
+                                     num_groups, partition_tokens);
     if (one_pass)
         *one_pass = op ? 1 : 0;
     if (prefix_partitions)
@@ -735,14 +751,15 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
     // asked for (partition_tokens < 0) or, automatically, when the groups'
     // CTAs alone fill the GPU; else the prefix is split into partitions.
     const int G = num_heads / num_kv_heads;
-    const int free_chunks = (batch + pkv::kPfRows / G - 1) / (pkv::kPfRows / G);
-    if ((int64_t)num_groups * plan.chunks > 65535)
+    const bool one_pass =
+        cascade_one_pass(batch, G, num_kv_heads, max_group_size, num_groups, partition_tokens);
+    if (!one_pass && (int64_t)num_groups * plan.chunks > 65535)
         return fail(PKV_ERR_UNSUPPORTED, "num_groups x member chunks (%lld) above 65535",
                     (long long)num_groups * plan.chunks);
-    const bool one_pass = cascade_one_pass(plan, batch, G, num_kv_heads, num_groups, partition_tokens);
     if (one_pass) {
+        const OnePassGrid og = one_pass_grid(batch, G, max_group_size, num_groups);
         CUtensorMap mq, mk4, mv4;
-        if ((s = make_query_map(&mq, query, batch, num_heads, head_dim, G, pkv::kPfRows / G, dtype)) != PKV_OK)
+        if ((s = make_query_map(&mq, query, batch, num_heads, head_dim, G, kOnePassRows / G, dtype)) != PKV_OK)
             return s;
         if ((s = make_cache_map_4d(&mk4, key_cache, num_blocks, block_size, num_kv_heads, head_dim,
                                    dtype)) != PKV_OK)
@@ -763,15 +780,15 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
         c.num_kv_heads = num_kv_heads;
         c.group = G;
         c.num_blocks = (int)num_blocks;
-        c.chunks = plan.chunks;
+        c.chunks = og.chunks;
         c.scale_log2 = scale_log2;
         c.suffix_tables = suffix_tables;
         c.suffix_lens = suffix_lens;
         c.out = static_cast<uint16_t *>(out);
         c.max_suffix_blocks = max_suffix_blocks;
         cudaError_t e = dtype == PKV_BF16
-                            ? dispatch_cascade_one_pass<true>(head_dim, block_size, mq, mk4, mv4, c, free_chunks, st)
-                            : dispatch_cascade_one_pass<false>(head_dim, block_size, mq, mk4, mv4, c, free_chunks, st);
+                            ? dispatch_cascade_one_pass<true>(head_dim, block_size, mq, mk4, mv4, c, og.free_chunks, st)
+                            : dispatch_cascade_one_pass<false>(head_dim, block_size, mq, mk4, mv4, c, og.free_chunks, st);
         if (e != cudaSuccess)
             return cuda_fail(e, "cascade_tc_kernel launch");
         return PKV_OK;

@@ -557,8 +557,8 @@ paged_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 // below complete the result, which equals the decode over the concatenated
 // table.  When there are enough groups to fill the GPU, one kernel does it all
 // instead (cascade_tc_kernel, pkv_prefill.cuh): a CTA per (kv head, chunk of
-// members) reads the group's whole prefix once and then each member's own
-// blocks, and writes the output rows; no records, no merge.
+// 32/G members) reads the group's whole prefix once and then each member's
+// own blocks, and writes the output rows; no records, no merge kernel.
 struct CascadeArgs {
     const uint16_t *query;           // [B, Hq, D]
     const int32_t *prefix_tables;    // [num_groups, max_prefix_blocks]

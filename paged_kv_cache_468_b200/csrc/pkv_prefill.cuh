@@ -80,6 +80,7 @@ constexpr int kPfThreads = 224;          // 7 warps
 constexpr uint32_t kPfTmemCols = 256;    // S/P: 2 x 64 columns, O: D columns at 128
 constexpr int kPfKStages = 3;
 constexpr int kPfVStages = 2;
+constexpr int kCasRows = 32;             // one-pass cascade: query rows per CTA (held 4 times)
 
 template <int D>
 struct PfShape {
@@ -112,7 +113,9 @@ enum PfBar {
     kBarVTail = 16,
     kBarDrain = 17,
     kBarTmemSlot = 18,   // not a barrier: the TMEM base address
-    kNumPfBars = 20
+    kBarEpi0 = 19,       // one-pass cascade: the softmax warps' partial results
+    kBarEpi1 = 20,
+    kNumPfBars = 22
 };
 // A barrier per S/P buffer completes once per two tiles, and buffer j & 1 is
 // refilled (S_{j+2}) only after P_j V_j has completed: no barrier can run two
@@ -128,7 +131,13 @@ enum TcMode : int {
     // the query rows of a group's members over the group's whole prefix, then
     // each member's rows over that member's own blocks (the other rows see
     // none of them); output rows.  Extra CTAs at the end of the grid take the
-    // sequences outside every group (own blocks only).
+    // sequences outside every group (own blocks only).  A CTA takes 32 query
+    // rows (32/G members) and holds them in all four softmax warps' lanes (Q
+    // is loaded four times): warp w weighs key columns 16w .. 16w+15 of every
+    // tile with its own running maximum and sum, so the four share the
+    // exponentials of a tile; their partial rows are merged by log-sum-exp in
+    // the epilogue.  The tensor core does the padding (M = 128 for 32 rows);
+    // the softmax, which bounds a tile's time, does none.
     kTcCascade = 2,
 };
 
@@ -167,8 +176,10 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
     const int lane = threadIdx.x & 31;
     constexpr bool kCas = MODE != kTcPrefill;   // a cascade mode: c, not a
     const int G = kCas ? c.group : a.group;
-    const int TT = kPfRows / G;   // query tokens (cascade: group members) per CTA
-    const int R = TT * G;         // rows in use (128 when G divides 128)
+    // query tokens (cascade: group members) per CTA; the one-pass cascade takes
+    // 32 query rows and holds them four times, once in each softmax warp's lanes
+    const int TT = (MODE == kTcCascade ? kCasRows : kPfRows) / G;
+    const int R = TT * G;         // rows in use (128, or 32 in the one pass, when G divides them)
     const int num_heads = kCas ? c.num_heads : a.num_heads;
     const int num_blocks = kCas ? c.num_blocks : a.num_blocks;
     const float scale_log2 = kCas ? c.scale_log2 : a.scale_log2;
@@ -192,6 +203,8 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         mbar_init(bar(kBarODone), 1);
         mbar_init(bar(kBarVTail), 1);
         mbar_init(bar(kBarDrain), 1);
+        mbar_init(bar(kBarEpi0), 4);            // one arrive per softmax warp
+        mbar_init(bar(kBarEpi1), 4);
         prefetch_tensormap(tm_q);
         prefetch_tensormap(tm_k);
         prefetch_tensormap(tm_v);
@@ -416,11 +429,14 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             // each is read once per group and kv head
             const uint64_t policy = kCas ? policy_evict_first() : policy_evict_normal();
             if (is_k && lane == 0) {
-                mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(Sh::kHalves * R * 128));
+                constexpr int kCopies = MODE == kTcCascade ? 4 : 1;   // row groups of 32
+                mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(kCopies * Sh::kHalves * R * 128));
 #pragma unroll
-                for (int h = 0; h < Sh::kHalves; ++h)
-                    tma_load_3d(sQ + h * Sh::kQHalf, tm_q, bar(kBarQFull), h * 64, kvh * G, q_tok0,
-                                policy);
+                for (int q = 0; q < kCopies; ++q)
+#pragma unroll
+                    for (int h = 0; h < Sh::kHalves; ++h)
+                        tma_load_3d(sQ + h * Sh::kQHalf + q * 32 * 128, tm_q, bar(kBarQFull), h * 64,
+                                    kvh * G, q_tok0, policy);
             }
             if constexpr (MODE == kTcCascade) {
                 if (!is_k) {
@@ -634,6 +650,183 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             tc_commit(bar(kBarDrain));
             mbar_wait_bounded(bar(kBarDrain), 0u, kWaitLimitNs);
         }
+    } else if constexpr (MODE == kTcCascade) {
+        // ---- one-pass cascade softmax: every softmax warp holds the CTA's
+        // query rows (up to 32: member rl / G, head rl % G) in its own lanes,
+        // and takes key columns 16w .. 16w+15 of every tile, with its own
+        // running maximum, sum and O rows; the four are merged at the end ----
+        const int rl = lane;
+        const bool real = rl < rows;
+        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int cw0 = warp * 16;                  // this warp's key columns
+        float m_used = kNegInf;
+        float l = 0.f;
+        bool ok = true;
+        const float sc = scale_log2;
+        const bool fold = sc > 0.f;
+        const float sm = fold ? 1.f : sc;
+        const float se = fold ? sc : 1.f;
+        Walk sw = walk_start();
+        for (int j = 0; j < nt; ++j) {
+            const int s = j & 1;
+            ok = mbar_wait_bounded(bar(kBarSFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
+            if (!__all_sync(0xffffffffu, ok)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            // valid key columns [clo, chi) and the rows [rlo, rhi) that see them
+            int clo = 0, chi, rlo = 0, rhi = rows;
+            const int nbs = (sw.len + BS - 1) / BS;
+            if (sw.m < 0) {
+                chi = min(kPfKeys, sw.len - sw.k * kPfKeys);
+            } else {
+                clo = sw.k == 0 ? nbs * BS - sw.len : 0;
+                chi = BS * min(BPT, nbs - sw.k * BPT);
+                rlo = sw.m * G;
+                rhi = rlo + G;
+            }
+            const int lo = max(clo, cw0), hi = min(chi, cw0 + 16);   // this warp's share
+            uint32_t pw[8];                         // packed weights of columns cw0 .. cw0+15
+            bool resc = false;
+            float alpha = 1.f;
+            if (lo < hi) {
+                uint32_t raw[16];
+                tmem_ld16(tmem + lane_base + s * kPfKeys + cw0, raw);
+                const bool row_on = rl >= rlo && rl < rhi;
+                float x[16];
+                float mx[4] = {kNegInf, kNegInf, kNegInf, kNegInf};
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float v = fold ? __uint_as_float(raw[i]) : __uint_as_float(raw[i]) * sm;
+                    x[i] = row_on && cw0 + i >= lo && cw0 + i < hi ? v : kNegInf;
+                    mx[i & 3] = fmaxf(mx[i & 3], x[i]);
+                }
+                const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * se;
+                resc = mt > m_used + 8.f;
+                const float m_new = resc ? mt : m_used;
+                alpha = resc ? ex2(m_used - m_new) : 1.f;
+                const float msub = m_new == kNegInf ? 0.f : m_new;
+                float rsv[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    pw[i] = pack2<BF16>(ex2(fmaf(x[2 * i], se, -msub)), ex2(fmaf(x[2 * i + 1], se, -msub)));
+                    const float2 pr = unpack2<BF16>(pw[i]);
+                    rsv[i & 3] += pr.x + pr.y;
+                }
+                l = l * alpha + ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3]));
+                m_used = m_new;
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    pw[i] = 0u;
+            }
+            if (j > 0) {
+                // as below: P_{j-1} V_{j-1} has completed before P_j is stored
+                ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+            }
+            if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tmem_ld32(tO + lane_base + c0, o);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tmem_st32(tO + lane_base + c0, o);
+                }
+            }
+            // P over the first 32 columns of S_j: this warp's 8 packed columns,
+            // zero for the other warps' keys
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                pk[i] = (i >> 3) == warp ? pw[i & 7] : 0u;
+            tmem_st32(tmem + lane_base + s * kPfKeys, pk);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar(kBarPFull + s));
+            walk_next(sw);
+        }
+        if (ok)
+            ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((nt - 1) & 1), kWaitLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok && lane == 0)
+            raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+        // merge the four warps' partial softmaxes of each row by log-sum-exp,
+        // through the K/V rings (free: every load has been consumed by an MMA
+        // that has completed); a warp that gave up leaves NaN as its maximum
+        float *st_m = reinterpret_cast<float *>(data + Sh::kKOff);   // [4][32]
+        float *st_l = st_m + 4 * 32;                                  // [4][32]
+        float *part = st_l + 4 * 32;                                  // [4][D][32], scaled O rows
+        st_m[warp * 32 + lane] = ok ? m_used : __int_as_float(0x7fc00000);
+        st_l[warp * 32 + lane] = l;
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(bar(kBarEpi0));
+        bool go = mbar_wait_bounded(bar(kBarEpi0), 0u, kWaitLimitNs);
+        float M = kNegInf;
+        bool bad = false;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float mw = st_m[w * 32 + lane];
+            bad |= mw != mw;
+            M = fmaxf(M, mw);
+        }
+        go = __all_sync(0xffffffffu, go && !bad);
+        if (go) {
+            float L = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                const float mw = st_m[w * 32 + lane];
+                L += mw == kNegInf ? 0.f : ex2(mw - M) * st_l[w * 32 + lane];
+            }
+            const float f = L > 0.f && m_used != kNegInf ? ex2(m_used - M) / L : 0.f;
+            tc_fence_after();
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + lane_base + c0, o);
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    part[(warp * D + c0 + i) * 32 + lane] = __uint_as_float(o[i]) * f;
+            }
+        }
+        __syncwarp();
+        if (lane == 0)
+            mbar_arrive(bar(kBarEpi1));
+        go = __all_sync(0xffffffffu, mbar_wait_bounded(bar(kBarEpi1), 0u, kWaitLimitNs) && go);
+        if (!go && lane == 0)
+            raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+        const int b = q_tok0 + rl / G;
+        if (go && real && (grouped || b < gs0 || b >= gsN)) {
+            // this warp writes columns D/4 * w .. D/4 * (w+1) - 1 of row rl
+            constexpr int CW = D / 4;
+            uint4 *orow = reinterpret_cast<uint4 *>(
+                c.out + ((size_t)b * num_heads + (size_t)kvh * G + rl % G) * D + warp * CW);
+#pragma unroll
+            for (int i = 0; i < CW; i += 8) {
+                uint32_t wd[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    float v0 = 0.f, v1 = 0.f;
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        v0 += part[(w * D + warp * CW + i + 2 * e) * 32 + lane];
+                        v1 += part[(w * D + warp * CW + i + 2 * e + 1) * 32 + lane];
+                    }
+                    wd[e] = pack2<BF16>(v0, v1);
+                }
+                orow[i / 8] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+        }
     } else {
         // ---- softmax and epilogue: thread = row r of the tile = TMEM lane r ----
         const int r = warp * 32 + lane;
@@ -650,7 +843,6 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         const bool fold = sc > 0.f;
         const float sm = fold ? 1.f : sc;       // applied before the maximum
         const float se = fold ? sc : 1.f;       // applied in the exponent
-        Walk sw = walk_start();                     // one-pass cascade: the tile walk
         for (int j = 0; j < nt; ++j) {
             const int s = j & 1;
             ok = mbar_wait_bounded(bar(kBarSFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
@@ -659,27 +851,6 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 break;
             }
             tc_fence_after();
-            // one-pass cascade: the tile's valid key columns [clo, chi) and the
-            // query rows [rlo, rhi) that see them (the prefix: every row; a
-            // member's own blocks: that member's G rows)
-            int clo = 0, chi = kPfKeys, rlo = 0, rhi = rows;
-            if constexpr (MODE == kTcCascade) {
-                const int nbs = (sw.len + BS - 1) / BS;
-                if (sw.m < 0) {
-                    chi = min(kPfKeys, sw.len - sw.k * kPfKeys);
-                } else {
-                    clo = sw.k == 0 ? nbs * BS - sw.len : 0;
-                    chi = BS * min(BPT, nbs - sw.k * BPT);
-                    rlo = sw.m * G;
-                    rhi = rlo + G;
-                }
-            }
-            // no row of this warp sees the tile: its weights are all zero
-            const bool warp_off = MODE == kTcCascade && (rhi <= warp * 32 || rlo >= warp * 32 + 32);
-            uint32_t pk[32];
-            bool resc = false;
-            float alpha = 1.f;
-            if (!warp_off) {
             uint32_t raw[64];
             tmem_ld64(tmem + lane_base + s * kPfKeys, raw);
             // eight independent max / sum chains, not 64-long ones
@@ -689,13 +860,7 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             for (int i = 0; i < 8; ++i)
                 mx[i] = kNegInf;
             const int t0 = j * kPfKeys;
-            bool all_visible;
-            if constexpr (MODE == kTcCascade)
-                all_visible = clo == 0 && chi == kPfKeys && rlo <= warp * 32 && rhi >= warp * 32 + 32;
-            else
-                all_visible = t0 + kPfKeys - 1 <= pos0;
-            const bool row_on = r >= rlo && r < rhi;
-            if (all_visible) {                      // every key visible to every row
+            if (t0 + kPfKeys - 1 <= pos0) {         // every key visible to every row
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     x[c] = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
@@ -705,23 +870,19 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const float v = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
-                    bool vis;
-                    if constexpr (MODE == kTcCascade)
-                        vis = row_on && c >= clo && c < chi;
-                    else
-                        vis = t0 + c <= pos;
-                    x[c] = vis ? v : kNegInf;
+                    x[c] = t0 + c <= pos ? v : kNegInf;
                     mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
             }
             const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                                    fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * se;
-            resc = mt > m_used + 8.f;               // first tile: m_used = -inf
+            const bool resc = mt > m_used + 8.f;    // first tile: m_used = -inf
             const float m_new = resc ? mt : m_used;
-            alpha = resc ? ex2(m_used - m_new) : 1.f;
+            const float alpha = resc ? ex2(m_used - m_new) : 1.f;
             const float msub = m_new == kNegInf ? 0.f : m_new;
             // the row sum is taken over the rounded weights the MMA multiplies,
             // so the normalised weights sum to one exactly
+            uint32_t pk[32];
             float rsv[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -735,11 +896,6 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
             l = l * alpha + rs;
             m_used = m_new;
-            } else {
-#pragma unroll
-                for (int c = 0; c < 32; ++c)
-                    pk[c] = 0u;
-            }
             if (j > 0) {
                 // Wait for P_{j-1} V_{j-1}: O then holds it (for the rescale),
                 // and O_DONE stays within one phase of this warp, so the
@@ -772,8 +928,6 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(bar(kBarPFull + s));
-            if constexpr (MODE == kTcCascade)
-                walk_next(sw);
         }
         if (ok)
             ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((nt - 1) & 1), kWaitLimitNs);
@@ -782,19 +936,13 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             const float inv = l > 0.f ? 1.f / l : 0.f;
             // query row (q_tok0 + r / G, head kvh * G + r % G): row0 is a multiple of G
             const size_t orow_i = (size_t)(q_tok0 + r / G) * num_heads + (size_t)kvh * G + r % G;
-            if constexpr (MODE != kTcPrefix) {
-                // one-pass cascade: only the rows of sequences this CTA covers
-                bool own = real;
-                if constexpr (MODE == kTcCascade) {
-                    const int b = q_tok0 + r / G;
-                    own = real && (grouped || b < gs0 || b >= gsN);
-                }
-                uint4 *orow = reinterpret_cast<uint4 *>((MODE == kTcPrefill ? a.out : c.out) + orow_i * D);
+            if constexpr (MODE == kTcPrefill) {
+                uint4 *orow = reinterpret_cast<uint4 *>(a.out + orow_i * D);
 #pragma unroll 1
                 for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t o[32];
                     tmem_ld32(tO + lane_base + c0, o);
-                    if (own) {
+                    if (real) {
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             uint32_t w[4];
