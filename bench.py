@@ -565,9 +565,25 @@ def read_ceiling(pkv, dev, stream, nbytes: int = 2 << 30, reps: int = 40) -> dic
             fn()
         ms = time_back_to_back(fn, reps, stream)
         rates[str(grid)] = round(nbytes / (ms * 1e-3) / 1e9, 1)
-    del buf
+    # the same bytes as 4 KiB chunks in a random order: a paged cache's blocks
+    # are scattered over the pool, and one kv head of one block (16 rows of a
+    # 128-wide head) is 4 KiB
+    chunk = 4096
+    order = torch.randperm(nbytes // chunk, generator=torch.Generator().manual_seed(5)).to(
+        torch.int32).to(dev)
+    gather = {}
+    for per_sm in (2, 4, 8):
+        grid = sms * per_sm
+        fn = lambda: pkv.hbm_gather_probe(buf, chunk, order, sink, grid)
+        for _ in range(3):
+            fn()
+        ms = time_back_to_back(fn, reps, stream)
+        gather[str(grid)] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+    del buf, order
     return {"gbs": max(rates.values()), "bytes": nbytes, "reps": reps, "by_grid": rates,
-            "kernel": "hbm_read_probe_kernel (16-byte ld.global.nc, 8 in flight per thread)"}
+            "kernel": "hbm_read_probe_kernel (16-byte ld.global.nc, 8 in flight per thread)",
+            "gather_4k_gbs": max(gather.values()), "gather_4k_by_grid": gather,
+            "gather_kernel": "hbm_gather_probe_kernel (4 KiB chunks in a random order, a warp per chunk)"}
 
 
 def roofline_entry(w: DecodeWorkload, t: dict, peaks: dict, ceiling) -> dict:
@@ -586,6 +602,8 @@ def roofline_entry(w: DecodeWorkload, t: dict, peaks: dict, ceiling) -> dict:
     if ceiling:
         r["read_ceiling_gbs"] = ceiling["gbs"]
         r["frac_of_read_ceiling"] = round(achieved / ceiling["gbs"], 4)
+        r["gather_ceiling_gbs"] = ceiling["gather_4k_gbs"]
+        r["frac_of_gather_ceiling"] = round(achieved / ceiling["gather_4k_gbs"], 4)
     return r
 
 

@@ -307,6 +307,14 @@ pkv_status pkv_paged_attention_decode_cascade(
  */
 pkv_status pkv_hbm_read_probe(const void *buf, size_t bytes, unsigned int *sink, int grid,
                               void *stream);
+/* hbm_gather_probe -- measurement only: reads a buffer of n_chunks chunks of
+ * chunk_bytes each (a multiple of 16), whole chunks in the order order[0 ..
+ * n_chunks) lists them (int32 chunk indices, device memory; an index outside
+ * the buffer is skipped), one warp per chunk.  With a random order of 4 KiB
+ * chunks this is the access pattern of a paged cache whose blocks are
+ * scattered over the pool.  Same alignment rules and errors as above. */
+pkv_status pkv_hbm_gather_probe(const void *buf, size_t chunk_bytes, const int32_t *order,
+                                int64_t n_chunks, unsigned int *sink, int grid, void *stream);
 
 /*
  * paged_attention_decode_static_workspace -- the same decode as

@@ -16,6 +16,7 @@ from .pagedkv import (  # noqa: F401
     decode_plan,
     decode_workspace_bytes,
     device_flags,
+    hbm_gather_probe,
     hbm_read_probe,
     kv_cache_write,
     lib,

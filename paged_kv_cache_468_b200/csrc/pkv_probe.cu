@@ -1,5 +1,6 @@
-// pkv_probe.cu -- a read-only HBM streaming kernel that measures the ceiling
-// the decode kernels are held against.
+// pkv_probe.cu -- read-only HBM kernels that measure the ceilings the decode
+// kernels are held against: a sequential stream, and whole chunks read in a
+// given (random) order.
 //
 // The decode path only reads its large inputs (K and V rows) and writes a
 // small output, so the copy bandwidth (read + write) is not its true upper
@@ -10,6 +11,7 @@
 
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cstdint>
 
 #include "pagedkv.h"
@@ -55,7 +57,63 @@ hbm_read_probe_kernel(const uint4 *__restrict__ buf, int64_t n_vec, uint32_t *__
         atomicXor(sink, acc);
 }
 
+// The same reads, as whole chunks taken in the order `order` lists them: a
+// warp reads one chunk at a time (its lanes' 16-byte loads across it, eight
+// in flight each), warps walking the list with a grid stride.  With a random
+// order of 4 KiB chunks this is the access a paged cache sees: blocks
+// scattered over the pool, each read whole once.
+__global__ void __launch_bounds__(kProbeThreads)
+hbm_gather_probe_kernel(const uint4 *__restrict__ buf, const int32_t *__restrict__ order,
+                        int64_t n_chunks, int64_t vec_per_chunk, uint32_t *__restrict__ sink)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t nw = (int64_t)gridDim.x * (kProbeThreads / 32);
+    uint32_t acc = 0;
+    for (int64_t c = ((int64_t)blockIdx.x * kProbeThreads + threadIdx.x) >> 5; c < n_chunks; c += nw) {
+        const int64_t ch = __ldg(order + c);
+        if (ch < 0 || ch >= n_chunks)
+            continue;                               // not a chunk of the buffer
+        const uint4 *src = buf + ch * vec_per_chunk;
+        for (int64_t v0 = lane; v0 < vec_per_chunk; v0 += 32 * kProbeUnroll) {
+            uint4 v[kProbeUnroll];
+#pragma unroll
+            for (int u = 0; u < kProbeUnroll; ++u)
+                v[u] = v0 + u * 32 < vec_per_chunk ? load_stream(src + v0 + u * 32) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+            for (int u = 0; u < kProbeUnroll; ++u)
+                acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+        }
+    }
+    acc = __reduce_xor_sync(0xffffffffu, acc);
+    if (lane == 0)
+        atomicXor(sink, acc);
+}
+
 }  // namespace
+
+extern "C" pkv_status pkv_hbm_gather_probe(const void *buf, size_t chunk_bytes, const int32_t *order,
+                                           int64_t n_chunks, unsigned int *sink, int grid, void *stream)
+{
+    if (!buf || !order || !sink || chunk_bytes == 0 || chunk_bytes % 16 != 0 || n_chunks <= 0 ||
+        n_chunks > INT32_MAX || grid <= 0 || grid > (1 << 20)) {
+        pkv_set_last_error("hbm_gather_probe: null pointer, chunk size not a positive multiple of 16, "
+                           "chunk count outside 1 .. 2^31-1, or grid outside 1 .. 2^20");
+        return PKV_ERR_INVALID_ARG;
+    }
+    if ((reinterpret_cast<uintptr_t>(buf) & 15u) || (reinterpret_cast<uintptr_t>(order) & 3u) ||
+        (reinterpret_cast<uintptr_t>(sink) & 3u)) {
+        pkv_set_last_error("hbm_gather_probe: buf must be 16-byte, order and sink 4-byte aligned");
+        return PKV_ERR_MISALIGNED;
+    }
+    hbm_gather_probe_kernel<<<(unsigned)grid, kProbeThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<const uint4 *>(buf), order, n_chunks, (int64_t)(chunk_bytes / 16), sink);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        pkv_set_last_error(cudaGetErrorString(e));
+        return PKV_ERR_CUDA;
+    }
+    return PKV_OK;
+}
 
 extern "C" pkv_status pkv_hbm_read_probe(const void *buf, size_t bytes, unsigned int *sink,
                                          int grid, void *stream)

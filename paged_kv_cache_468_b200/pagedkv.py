@@ -109,6 +109,8 @@ def lib() -> ctypes.CDLL:
                                                i32, pint, pint]
         L.pkv_hbm_read_probe.restype = i32
         L.pkv_hbm_read_probe.argtypes = [P, sz, P, i32, P]
+        L.pkv_hbm_gather_probe.restype = i32
+        L.pkv_hbm_gather_probe.argtypes = [P, sz, P, i64, P, i32, P]
         _lib = L
         return L
 
@@ -199,6 +201,20 @@ def hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, grid: int,
     _check(lib().pkv_hbm_read_probe(_dev(buf, "buf"), buf.numel() * buf.element_size(),
                                     _dev(sink, "sink"), int(grid), _stream_handle(stream, buf.device)),
            "pkv_hbm_read_probe")
+
+
+def hbm_gather_probe(buf: torch.Tensor, chunk_bytes: int, order: torch.Tensor, sink: torch.Tensor,
+                     grid: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Read `buf` as whole chunks of chunk_bytes in the order `order` (int32 CUDA
+    tensor of chunk indices) lists them; measurement of the paged-read ceiling."""
+    if order.dtype != torch.int32 or not order.is_cuda or sink.dtype != torch.int32:
+        raise ValueError("order and sink must be int32 CUDA tensors")
+    n = (buf.numel() * buf.element_size()) // int(chunk_bytes)
+    if order.numel() != n:
+        raise ValueError("order must list every chunk of buf once")
+    _check(lib().pkv_hbm_gather_probe(_dev(buf, "buf"), int(chunk_bytes), _dev(order, "order"), n,
+                                      _dev(sink, "sink"), int(grid), _stream_handle(stream, buf.device)),
+           "pkv_hbm_gather_probe")
 
 
 def kv_cache_write(key: torch.Tensor, value: torch.Tensor, slot_mapping: torch.Tensor,

@@ -197,3 +197,13 @@ def test_cascade_plan_choice():
     assert pkv.decode_cascade_plan(96, 32, 8, 128, 125, 16, 8, 0, 16, -1) == (False, 4)   # no groups
     with pytest.raises(pkv.PagedKVError):
         pkv.decode_cascade_plan(96, 32, 8, 128, 125, 16, 8, 97, 16, 0)                     # > batch
+
+
+def test_hbm_gather_probe_host_validation():
+    L = pkv.lib()
+    a16 = 0x10000
+    assert L.pkv_hbm_gather_probe(None, 4096, a16, 4, a16, 1, None) == pagedkv.ERR_INVALID_ARG
+    assert L.pkv_hbm_gather_probe(a16, 4095, a16, 4, a16, 1, None) == pagedkv.ERR_INVALID_ARG
+    assert L.pkv_hbm_gather_probe(a16, 4096, a16, 0, a16, 1, None) == pagedkv.ERR_INVALID_ARG
+    assert L.pkv_hbm_gather_probe(a16 + 8, 4096, a16, 4, a16, 1, None) == pagedkv.ERR_MISALIGNED
+    assert L.pkv_hbm_gather_probe(a16, 4096, a16 + 2, 4, a16, 1, None) == pagedkv.ERR_MISALIGNED
