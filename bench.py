@@ -103,7 +103,8 @@ _CASCADE_CODE = [
     ("pkv_kernels.cuh", ["CascadeArgs", "load_slice", "lse_merge_cascade_kernel"]),
     ("pkv_prefill.cuh", ["PrefillArgs", "PfShape", "PfBar", "TcMode", "tc_attend", "prefix_tc_kernel",
                          "cascade_tc_kernel"]),
-    ("pagedkv.cu", ["make_query_map", "make_cache_map_4d", "cascade_plan", "launch_prefix",
+    ("pagedkv.cu", ["make_query_map", "make_cache_map_4d", "CacheMaps", "make_cache_maps", "cascade_plan",
+                    "launch_prefix",
                     "dispatch_prefix", "launch_cascade_one_pass", "dispatch_cascade_one_pass",
                     "cascade_one_pass", "pkv_paged_attention_decode_cascade"]),
 ]

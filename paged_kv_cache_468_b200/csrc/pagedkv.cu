@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -44,6 +45,22 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 constexpr int kPlanSmCount = 148;        // B200 SM count used by the automatic plan
+// A prefill CTA takes up to this many row tiles (of 128/G query tokens) of one
+// (sequence, kv head) in turn: fewer CTAs amortise their set-up over more
+// tiles, but each CTA's work grows, and the hardware's balancing of CTAs over
+// the SMs needs the largest CTA to stay small next to the average work per SM.
+constexpr int kPrefillMaxTilesPerCta = 4;
+
+int prefill_tiles_per_cta(int batch, int Hkv, int row_tiles, int sms)
+{
+    // at most 1/8 of the average work per CTA slot (2 per SM) in one CTA,
+    // counting a row tile's work at half the largest one's
+    const int64_t per_slot_share = (int64_t)batch * Hkv * row_tiles / (2 * 2 * 8 * (int64_t)sms);
+    int t = 1;
+    while (t * 2 <= kPrefillMaxTilesPerCta && t * 2 <= per_slot_share)
+        t *= 2;
+    return t;
+}
 constexpr int kAutoPartitionTokens = 512;
 
 // ---- TMA tensor maps ------------------------------------------------------
@@ -111,6 +128,24 @@ pkv_status make_cache_map_4d(CUtensorMap *map, const void *base, int64_t num_blo
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled (4-D cache) failed (CUresult %d)", (int)r);
+    return PKV_OK;
+}
+
+// K and V caches, each as the 3-D view (whole blocks) and the 4-D view
+// (shifted partly filled blocks) the tensor-core kernels load through.
+struct CacheMaps {
+    CUtensorMap k, v, k4, v4;
+};
+
+pkv_status make_cache_maps(CacheMaps *m, const void *key_cache, const void *value_cache,
+                           int64_t num_blocks, int bs, int Hkv, int D, pkv_dtype dt)
+{
+    pkv_status s;
+    if ((s = make_cache_map(&m->k, key_cache, num_blocks, bs, Hkv, D, dt)) != PKV_OK ||
+        (s = make_cache_map(&m->v, value_cache, num_blocks, bs, Hkv, D, dt)) != PKV_OK ||
+        (s = make_cache_map_4d(&m->k4, key_cache, num_blocks, bs, Hkv, D, dt)) != PKV_OK ||
+        (s = make_cache_map_4d(&m->v4, value_cache, num_blocks, bs, Hkv, D, dt)) != PKV_OK)
+        return s;
     return PKV_OK;
 }
 
@@ -579,7 +614,7 @@ pkv_status cascade_plan(int batch, int Hq, int Hkv, int D, int max_prefix_blocks
 }
 
 template <int D, int BS, bool BF16>
-cudaError_t launch_prefix(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+cudaError_t launch_prefix(const CUtensorMap &mq, const CacheMaps &cm,
                           const pkv::CascadeArgs &c, cudaStream_t st)
 {
     constexpr int smem = pkv::PfShape<D>::kSmemBytes;
@@ -592,23 +627,23 @@ cudaError_t launch_prefix(const CUtensorMap &mq, const CUtensorMap &mk, const CU
         return e;
     const dim3 grid((unsigned)c.num_parts, (unsigned)c.num_kv_heads,
                     (unsigned)((size_t)c.num_groups * c.chunks));
-    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, mk, mv, c);
+    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, cm.k, cm.v, cm.k4, cm.v4, c);
 }
 
 template <bool BF16>
-cudaError_t dispatch_prefix(int D, int bs, const CUtensorMap &mq, const CUtensorMap &mk,
-                            const CUtensorMap &mv, const pkv::CascadeArgs &c, cudaStream_t st)
+cudaError_t dispatch_prefix(int D, int bs, const CUtensorMap &mq, const CacheMaps &cm,
+                            const pkv::CascadeArgs &c, cudaStream_t st)
 {
-    if (D == 64 && bs == 16) return launch_prefix<64, 16, BF16>(mq, mk, mv, c, st);
-    if (D == 64 && bs == 32) return launch_prefix<64, 32, BF16>(mq, mk, mv, c, st);
-    if (D == 128 && bs == 16) return launch_prefix<128, 16, BF16>(mq, mk, mv, c, st);
-    return launch_prefix<128, 32, BF16>(mq, mk, mv, c, st);
+    if (D == 64 && bs == 16) return launch_prefix<64, 16, BF16>(mq, cm, c, st);
+    if (D == 64 && bs == 32) return launch_prefix<64, 32, BF16>(mq, cm, c, st);
+    if (D == 128 && bs == 16) return launch_prefix<128, 16, BF16>(mq, cm, c, st);
+    return launch_prefix<128, 32, BF16>(mq, cm, c, st);
 }
 
 // One-pass cascade: a CTA per (kv head, chunk of 32/G members of a group),
 // then free_chunks CTAs per kv head for the sequences outside every group.
 template <int D, int BS, bool BF16>
-cudaError_t launch_cascade_one_pass(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+cudaError_t launch_cascade_one_pass(const CUtensorMap &mq, const CacheMaps &cm,
                                     const pkv::CascadeArgs &c, int free_chunks, cudaStream_t st)
 {
     constexpr int smem = pkv::PfShape<D>::kSmemBytes;
@@ -621,18 +656,17 @@ cudaError_t launch_cascade_one_pass(const CUtensorMap &mq, const CUtensorMap &mk
         return e;
     const dim3 grid(1u, (unsigned)c.num_kv_heads,
                     (unsigned)((size_t)c.num_groups * c.chunks + (size_t)free_chunks));
-    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, mk, mv, c);
+    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, cm.k, cm.v, cm.k4, cm.v4, c);
 }
 
 template <bool BF16>
-cudaError_t dispatch_cascade_one_pass(int D, int bs, const CUtensorMap &mq, const CUtensorMap &mk,
-                                      const CUtensorMap &mv, const pkv::CascadeArgs &c,
-                                      int free_chunks, cudaStream_t st)
+cudaError_t dispatch_cascade_one_pass(int D, int bs, const CUtensorMap &mq, const CacheMaps &cm,
+                                      const pkv::CascadeArgs &c, int free_chunks, cudaStream_t st)
 {
-    if (D == 64 && bs == 16) return launch_cascade_one_pass<64, 16, BF16>(mq, mk, mv, c, free_chunks, st);
-    if (D == 64 && bs == 32) return launch_cascade_one_pass<64, 32, BF16>(mq, mk, mv, c, free_chunks, st);
-    if (D == 128 && bs == 16) return launch_cascade_one_pass<128, 16, BF16>(mq, mk, mv, c, free_chunks, st);
-    return launch_cascade_one_pass<128, 32, BF16>(mq, mk, mv, c, free_chunks, st);
+    if (D == 64 && bs == 16) return launch_cascade_one_pass<64, 16, BF16>(mq, cm, c, free_chunks, st);
+    if (D == 64 && bs == 32) return launch_cascade_one_pass<64, 32, BF16>(mq, cm, c, free_chunks, st);
+    if (D == 128 && bs == 16) return launch_cascade_one_pass<128, 16, BF16>(mq, cm, c, free_chunks, st);
+    return launch_cascade_one_pass<128, 32, BF16>(mq, cm, c, free_chunks, st);
 }
 
 }  // namespace
@@ -758,14 +792,11 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
                     (long long)num_groups * plan.chunks);
     if (one_pass) {
         const OnePassGrid og = one_pass_grid(batch, G, max_group_size, num_groups);
-        CUtensorMap mq, mk4, mv4;
-        if ((s = make_query_map(&mq, query, batch, num_heads, head_dim, G, kOnePassRows / G, dtype)) != PKV_OK)
-            return s;
-        if ((s = make_cache_map_4d(&mk4, key_cache, num_blocks, block_size, num_kv_heads, head_dim,
-                                   dtype)) != PKV_OK)
-            return s;
-        if ((s = make_cache_map_4d(&mv4, value_cache, num_blocks, block_size, num_kv_heads, head_dim,
-                                   dtype)) != PKV_OK)
+        CUtensorMap mq;
+        CacheMaps cm;
+        if ((s = make_query_map(&mq, query, batch, num_heads, head_dim, G, kOnePassRows / G, dtype)) != PKV_OK ||
+            (s = make_cache_maps(&cm, key_cache, value_cache, num_blocks, block_size, num_kv_heads,
+                                 head_dim, dtype)) != PKV_OK)
             return s;
         pkv::CascadeArgs c{};
         c.query = static_cast<const uint16_t *>(query);
@@ -787,8 +818,8 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
         c.out = static_cast<uint16_t *>(out);
         c.max_suffix_blocks = max_suffix_blocks;
         cudaError_t e = dtype == PKV_BF16
-                            ? dispatch_cascade_one_pass<true>(head_dim, block_size, mq, mk4, mv4, c, og.free_chunks, st)
-                            : dispatch_cascade_one_pass<false>(head_dim, block_size, mq, mk4, mv4, c, og.free_chunks, st);
+                            ? dispatch_cascade_one_pass<true>(head_dim, block_size, mq, cm, c, og.free_chunks, st)
+                            : dispatch_cascade_one_pass<false>(head_dim, block_size, mq, cm, c, og.free_chunks, st);
         if (e != cudaSuccess)
             return cuda_fail(e, "cascade_tc_kernel launch");
         return PKV_OK;
@@ -823,8 +854,12 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
         if ((s = make_query_map(&mq, query, batch, num_heads, head_dim, c.group,
                                 pkv::kPfRows / c.group, dtype)) != PKV_OK)
             return s;
-        e = dtype == PKV_BF16 ? dispatch_prefix<true>(head_dim, block_size, mq, mk, mv, c, st)
-                              : dispatch_prefix<false>(head_dim, block_size, mq, mk, mv, c, st);
+        CacheMaps cm;
+        if ((s = make_cache_maps(&cm, key_cache, value_cache, num_blocks, block_size, num_kv_heads,
+                                 head_dim, dtype)) != PKV_OK)
+            return s;
+        e = dtype == PKV_BF16 ? dispatch_prefix<true>(head_dim, block_size, mq, cm, c, st)
+                              : dispatch_prefix<false>(head_dim, block_size, mq, cm, c, st);
         if (e != cudaSuccess)
             return cuda_fail(e, "prefix_tc_kernel launch");
     }
@@ -879,7 +914,7 @@ extern "C" pkv_status pkv_paged_attention_decode_cascade(
 namespace {
 
 template <int D, int BS, bool BF16>
-cudaError_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+cudaError_t launch_prefill(const CUtensorMap &mq, const CacheMaps &cm,
                            const pkv::PrefillArgs &p, int max_query_len, cudaStream_t st)
 {
     constexpr int smem = pkv::PfShape<D>::kSmemBytes;
@@ -890,21 +925,28 @@ cudaError_t launch_prefill(const CUtensorMap &mq, const CUtensorMap &mk, const C
                                  cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess)
         return e;
+    // a CTA per (tiles_per_cta row tiles, kv head, sequence)
     const int tokens_per_cta = pkv::kPfRows / p.group;
-    const dim3 grid((unsigned)((max_query_len + tokens_per_cta - 1) / tokens_per_cta),
+    const int row_tiles = (max_query_len + tokens_per_cta - 1) / tokens_per_cta;
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, current_device());
+    if (e != cudaSuccess)
+        return e;
+    pkv::PrefillArgs q = p;
+    q.tiles_per_cta = prefill_tiles_per_cta(p.batch, p.num_kv_heads, row_tiles, std::max(sms, 1));
+    const dim3 grid((unsigned)((row_tiles + q.tiles_per_cta - 1) / q.tiles_per_cta),
                     (unsigned)p.num_kv_heads, (unsigned)p.batch);
-    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, mk, mv, p);
+    return launch_pdl(kern, grid, dim3(pkv::kPfThreads), smem, st, mq, cm.k, cm.v, cm.k4, cm.v4, q);
 }
 
 template <bool BF16>
-cudaError_t dispatch_prefill(int D, int bs, const CUtensorMap &mq, const CUtensorMap &mk,
-                             const CUtensorMap &mv, const pkv::PrefillArgs &p, int max_query_len,
-                             cudaStream_t st)
+cudaError_t dispatch_prefill(int D, int bs, const CUtensorMap &mq, const CacheMaps &cm,
+                             const pkv::PrefillArgs &p, int max_query_len, cudaStream_t st)
 {
-    if (D == 64 && bs == 16) return launch_prefill<64, 16, BF16>(mq, mk, mv, p, max_query_len, st);
-    if (D == 64 && bs == 32) return launch_prefill<64, 32, BF16>(mq, mk, mv, p, max_query_len, st);
-    if (D == 128 && bs == 16) return launch_prefill<128, 16, BF16>(mq, mk, mv, p, max_query_len, st);
-    return launch_prefill<128, 32, BF16>(mq, mk, mv, p, max_query_len, st);
+    if (D == 64 && bs == 16) return launch_prefill<64, 16, BF16>(mq, cm, p, max_query_len, st);
+    if (D == 64 && bs == 32) return launch_prefill<64, 32, BF16>(mq, cm, p, max_query_len, st);
+    if (D == 128 && bs == 16) return launch_prefill<128, 16, BF16>(mq, cm, p, max_query_len, st);
+    return launch_prefill<128, 32, BF16>(mq, cm, p, max_query_len, st);
 }
 
 }  // namespace
@@ -938,14 +980,13 @@ extern "C" pkv_status pkv_paged_attention_prefill(
         return fail(PKV_ERR_INVALID_ARG, "null pointer");
     if (!aligned16(query) || !aligned16(key_cache) || !aligned16(value_cache) || !aligned16(out))
         return fail(PKV_ERR_MISALIGNED, "query/cache/out pointers must be 16-byte aligned");
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq;
+    CacheMaps cm;
     const int group = num_heads / num_kv_heads;
     if ((s = make_query_map(&mq, query, num_tokens, num_heads, head_dim, group, pkv::kPfRows / group,
-                            dtype)) != PKV_OK)
-        return s;
-    if ((s = make_cache_map(&mk, key_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
-        return s;
-    if ((s = make_cache_map(&mv, value_cache, num_blocks, block_size, num_kv_heads, head_dim, dtype)) != PKV_OK)
+                            dtype)) != PKV_OK ||
+        (s = make_cache_maps(&cm, key_cache, value_cache, num_blocks, block_size, num_kv_heads, head_dim,
+                             dtype)) != PKV_OK)
         return s;
     pkv::PrefillArgs p;
     p.query = static_cast<const uint16_t *>(query);
@@ -964,8 +1005,8 @@ extern "C" pkv_status pkv_paged_attention_prefill(
     p.scale_log2 = (float)((double)scale * 1.4426950408889634);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e = dtype == PKV_BF16
-                        ? dispatch_prefill<true>(head_dim, block_size, mq, mk, mv, p, max_query_len, st)
-                        : dispatch_prefill<false>(head_dim, block_size, mq, mk, mv, p, max_query_len, st);
+                        ? dispatch_prefill<true>(head_dim, block_size, mq, cm, p, max_query_len, st)
+                        : dispatch_prefill<false>(head_dim, block_size, mq, cm, p, max_query_len, st);
     if (e != cudaSuccess)
         return cuda_fail(e, "prefill_tc_kernel launch");
     return PKV_OK;

@@ -12,10 +12,10 @@
 // section 三); query token i sits at position L_b - C_b + i and attends
 // causally over tokens 0 .. L_b - C_b + i of its paged cache.
 //
-// One CTA per (row tile, kv head, sequence); for the prefix pass, per
-// (prefix partition, kv head, chunk of 128/G group members).  A row is a
-// (query token or group member, head of the kv head's GQA group) pair, 128
-// rows per CTA (the M of every MMA).
+// A prefill CTA takes 1-4 consecutive row tiles of one (kv head, sequence);
+// the prefix pass one CTA per (prefix partition, kv head, chunk of 128/G group
+// members).  A row is a (query token or group member, head of the kv head's
+// GQA group) pair, 128 rows per tile (the M of every MMA).
 // Keys are taken 64 at a time (a "key tile": 64 / block_size cache blocks
 // located through the block table, exactly as the decode kernels do):
 //
@@ -46,11 +46,16 @@
 //   * While P_j is stored, the only MMA that can be running is S_{j+1}, which
 //     writes the other buffer.
 // Warp roles: 0-3 softmax + epilogue (warp w owns TMEM lanes 32w..32w+31),
-// 4 loads Q and the K ring (3 stages), 5 allocates TMEM and issues every MMA,
-// 6 loads the V ring (2 stages) and clears V rows past the last visible key
-// (so masked weights meet finite values).  Every wait is bounded; on a time-out
-// the CTA records PKV_DEVFLAG_WAIT_TIMEOUT, lets in-flight copies and MMAs
-// finish and frees its TMEM.
+// 4 loads the K ring (3 stages), 5 allocates TMEM and issues every MMA, 6
+// loads the V ring (2 stages), 7 loads Q.  Whole blocks come through a 3-D
+// view of the cache; a sequence's partly filled last block comes through a
+// 4-D view {head_dim, kv heads, block rows, blocks} at a negative row offset,
+// so that the cells past its end are never read (the rows before it read as
+// zero) and a masked key always meets a finite V row.  A prefill CTA takes a few
+// consecutive row tiles of one (sequence, kv head) in turn; the other modes
+// run one work tile per CTA.  Every wait is bounded; on a time-out the CTA
+// records PKV_DEVFLAG_WAIT_TIMEOUT, lets in-flight copies and MMAs finish and
+// frees its TMEM.
 #pragma once
 
 #include "pkv_kernels.cuh"
@@ -71,12 +76,13 @@ struct PrefillArgs {
     int num_kv_heads;
     int group;
     int num_blocks;
+    int tiles_per_cta;               // consecutive row tiles (of 128/G query tokens) a CTA takes
     float scale_log2;
 };
 
 constexpr int kPfRows = 128;             // query rows per CTA (MMA M)
 constexpr int kPfKeys = 64;              // keys per tile (N of Q K^T, K of P V)
-constexpr int kPfThreads = 224;          // 7 warps
+constexpr int kPfThreads = 256;          // 8 warps
 constexpr uint32_t kPfTmemCols = 256;    // S/P: 2 x 64 columns, O: D columns at 128
 constexpr int kPfKStages = 3;
 constexpr int kPfVStages = 2;
@@ -110,16 +116,27 @@ enum PfBar {
     kBarSFull = 11,    // 2, one per S/P buffer
     kBarPFull = 13,    // 2, one per S/P buffer
     kBarODone = 15,
-    kBarVTail = 16,
-    kBarDrain = 17,
-    kBarTmemSlot = 18,   // not a barrier: the TMEM base address
-    kBarEpi0 = 19,       // one-pass cascade: the softmax warps' partial results
-    kBarEpi1 = 20,
+    kBarDrain = 16,
+    kBarTmemSlot = 17,   // not a barrier: the TMEM base address
+    kBarEpi0 = 18,       // one-pass cascade: the softmax warps' partial results
+    kBarEpi1 = 19,
+    kBarQEmpty = 20,     // the Q buffer is free: the work tile's last S has completed
     kNumPfBars = 22
 };
 // A barrier per S/P buffer completes once per two tiles, and buffer j & 1 is
 // refilled (S_{j+2}) only after P_j V_j has completed: no barrier can run two
 // phases ahead of its waiter.
+
+// Bits lo .. hi-1 of a 64-column mask (clamped to 0 .. 64; empty when hi <= lo).
+__device__ __forceinline__ uint64_t col_range(int lo, int hi)
+{
+    lo = max(lo, 0);
+    hi = min(hi, 64);
+    if (hi <= lo)
+        return 0ull;
+    const uint64_t upto = hi >= 64 ? ~0ull : (1ull << hi) - 1ull;
+    return upto & ~((1ull << lo) - 1ull);
+}
 
 // What a CTA of the shared body computes.
 enum TcMode : int {
@@ -151,7 +168,8 @@ enum TcMode : int {
 // The body shared by the three modes.
 template <int D, int BS, bool BF16, int MODE>
 __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtensorMap *tm_k,
-                                          const CUtensorMap *tm_v, const PrefillArgs &a,
+                                          const CUtensorMap *tm_v, const CUtensorMap *tm_k4,
+                                          const CUtensorMap *tm_v4, const PrefillArgs &a,
                                           const CascadeArgs &c)
 {
     using Sh = PfShape<D>;
@@ -201,13 +219,15 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         mbar_init(bar(kBarPFull + 0), 4);       // one arrive per softmax warp
         mbar_init(bar(kBarPFull + 1), 4);
         mbar_init(bar(kBarODone), 1);
-        mbar_init(bar(kBarVTail), 1);
+        mbar_init(bar(kBarQEmpty), 1);
         mbar_init(bar(kBarDrain), 1);
         mbar_init(bar(kBarEpi0), 4);            // one arrive per softmax warp
         mbar_init(bar(kBarEpi1), 4);
         prefetch_tensormap(tm_q);
         prefetch_tensormap(tm_k);
         prefetch_tensormap(tm_v);
+        prefetch_tensormap(tm_k4);
+        prefetch_tensormap(tm_v4);
     }
     fence_mbar_init();
     __syncthreads();
@@ -230,30 +250,8 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
     bool grouped = false;
     int mlen[4] = {0, 0, 0, 0};
     if constexpr (MODE == kTcPrefill) {
-        const int tile = blockIdx.x;
-        const int b = blockIdx.z;
-        const int q0 = __ldg(a.query_start + b);
-        int C = __ldg(a.query_start + b + 1) - q0;
-        int L = __ldg(a.context_lens + b);
-        const int span = a.max_blocks * BS;
-        if (q0 < 0 || C < 0 || q0 + C > a.num_tokens || C > a.max_query_len || L < 0 || L > span ||
-            C > L) {
-            if (threadIdx.x == 0 && tile == 0 && kvh == 0)
-                raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
-            L = L < 0 ? 0 : (L > span ? span : L);
-            if (q0 < 0 || C < 0 || q0 + C > a.num_tokens)
-                C = 0;                              // rows outside query/out: skip the sequence
-            C = min(C, min(L, a.max_query_len));
-        }
-        rows = C * G;
-        row0 = tile * R;
-        if (row0 >= rows)
-            return;                                 // whole CTA, before TMEM is touched
-        const int i0 = tile * TT;                   // first query token of the CTA
-        q_tok0 = q0 + i0;
-        pos0 = L - C + i0;                          // the first row's last key
-        p_max = L - C + min(C, i0 + TT) - 1;        // last key any row of the CTA sees
-        trow = a.block_tables + (size_t)b * a.max_blocks;
+        rows = row0 = q_tok0 = p_max = pos0 = 0;   // per work tile: next_work below
+        trow = a.block_tables;
     } else if constexpr (MODE == kTcPrefix) {
         const int pp = blockIdx.x;
         const int g = blockIdx.z / c.chunks;
@@ -398,6 +396,79 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
     const int nt = MODE == kTcCascade ? nt_cas : p_max / kPfKeys + 1;   // key tiles
     const int nblk = p_max / BS + 1;                // cache blocks read (other modes)
 
+    // Work tiles.  A prefill CTA takes tiles_per_cta consecutive row tiles of
+    // one (sequence, kv head), the last (longest: most keys) first.  Its
+    // tensor memory, rings and barrier phases carry over from tile to tile,
+    // and the next tile's Q and first keys load while the current one
+    // finishes; the CTAs of one (sequence, kv head) run side by side, so their
+    // common keys come from L2.  The other modes run the one tile set up above.
+    struct Wk {
+        int rows, row0, q_tok0, p_max, pos0, kvh, nt, nblk;
+        int tail;    // valid rows of block nblk-1 when it is the sequence's partly filled last block, else 0
+        const int32_t *trow;
+    };
+    // prefill: the sequence's chunk, read once per CTA
+    int pf_rt = 0, pf_q0 = 0, pf_C = 0, pf_L = 0;
+    if constexpr (MODE == kTcPrefill) {
+        const int b = blockIdx.z;
+        pf_q0 = __ldg(a.query_start + b);
+        pf_C = __ldg(a.query_start + b + 1) - pf_q0;
+        pf_L = __ldg(a.context_lens + b);
+        const int span = a.max_blocks * BS;
+        if (pf_q0 < 0 || pf_C < 0 || pf_q0 + pf_C > a.num_tokens || pf_C > a.max_query_len || pf_L < 0 ||
+            pf_L > span || pf_C > pf_L) {
+            if (threadIdx.x == 0 && blockIdx.x == 0 && blockIdx.y == 0)
+                raise_flag(PKV_DEVFLAG_CONTEXT_RANGE);
+            pf_L = pf_L < 0 ? 0 : (pf_L > span ? span : pf_L);
+            if (pf_q0 < 0 || pf_C < 0 || pf_q0 + pf_C > a.num_tokens)
+                pf_C = 0;                           // rows outside query/out: skip the sequence
+            pf_C = min(pf_C, min(pf_L, a.max_query_len));
+        }
+        // the CTA's row tiles that hold query tokens, last first
+        const int rt_lo = blockIdx.x * a.tiles_per_cta;
+        pf_rt = min((pf_C + TT - 1) / TT, rt_lo + a.tiles_per_cta) - 1;
+        if (pf_rt < rt_lo)
+            return;                                 // the chunk ends before this CTA's tiles
+    }
+    bool single_done = false;
+    auto next_work = [&](Wk &wk) -> bool {
+        if constexpr (MODE == kTcPrefill) {
+            if (pf_rt < (int)blockIdx.x * a.tiles_per_cta)
+                return false;
+            const int rt = pf_rt--;
+            const int i0 = rt * TT;                 // first query token of the tile
+            wk.rows = pf_C * G;
+            wk.row0 = rt * R;
+            wk.q_tok0 = pf_q0 + i0;
+            wk.pos0 = pf_L - pf_C + i0;             // the first row's last key
+            wk.p_max = pf_L - pf_C + min(pf_C, i0 + TT) - 1;   // last key any row of the tile sees
+            wk.kvh = blockIdx.y;
+            wk.nt = wk.p_max / kPfKeys + 1;
+            wk.nblk = wk.p_max / BS + 1;
+            wk.tail = (pf_L % BS != 0 && (pf_L - 1) / BS == wk.nblk - 1) ? pf_L % BS : 0;
+            wk.trow = a.block_tables + (size_t)blockIdx.z * a.max_blocks;
+            return true;
+        } else {
+            if (single_done)
+                return false;
+            single_done = true;
+            // prefix partitions are whole blocks
+            wk = Wk{rows, row0, q_tok0, p_max, pos0, kvh, nt, nblk, 0, trow};
+            return true;
+        }
+    };
+
+    // Keys outside a tile's valid range meet V rows with weight 0, so those
+    // rows must be finite: the V ring starts at zero and then only ever holds
+    // loaded rows -- never a cell past a sequence's end (a partly filled last
+    // block is loaded shifted, the rows before it read as zero) -- or zero fill.
+    {
+        uint4 *vr = reinterpret_cast<uint4 *>(data + Sh::kVOff);
+        for (int i = threadIdx.x; i < kPfVStages * Sh::kKVBytes / 16; i += kPfThreads)
+            vr[i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();   // before any TMA write of the ring (ordered by the barrier below)
+    }
+
     // ---- tensor memory ----
     if (warp == 5) {
         tmem_alloc(bar(kBarTmemSlot), kPfTmemCols);
@@ -416,7 +487,8 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
     if (warp == 4 || warp == 6) {
         // ---- loads: warp 4 Q and the K ring, warp 6 the V ring ----
         const bool is_k = warp == 4;
-        const CUtensorMap *tm = is_k ? tm_k : tm_v;
+        const CUtensorMap *tm = is_k ? tm_k : tm_v;        // 3-D view: whole blocks
+        const CUtensorMap *tm4 = is_k ? tm_k4 : tm_v4;     // 4-D view: shifted last blocks
         const int full0 = is_k ? kBarKFull : kBarVFull;
         const int empty0 = is_k ? kBarKEmpty : kBarVEmpty;
         const uint32_t ring = is_k ? sK : sV;
@@ -428,27 +500,7 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             // prefill: the sequence's other CTAs reread these blocks; cascade:
             // each is read once per group and kv head
             const uint64_t policy = kCas ? policy_evict_first() : policy_evict_normal();
-            if (is_k && lane == 0) {
-                constexpr int kCopies = MODE == kTcCascade ? 4 : 1;   // row groups of 32
-                mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(kCopies * Sh::kHalves * R * 128));
-#pragma unroll
-                for (int q = 0; q < kCopies; ++q)
-#pragma unroll
-                    for (int h = 0; h < Sh::kHalves; ++h)
-                        tma_load_3d(sQ + h * Sh::kQHalf + q * 32 * 128, tm_q, bar(kBarQFull), h * 64,
-                                    kvh * G, q_tok0, policy);
-            }
             if constexpr (MODE == kTcCascade) {
-                if (!is_k) {
-                    // keys outside a tile's valid columns meet these V rows with
-                    // weight 0, so they must be finite: the ring starts at zero
-                    // and then only holds loaded rows or rows read as zero
-                    uint4 *vr = reinterpret_cast<uint4 *>(data + Sh::kVOff);
-                    for (int i = lane; i < kPfVStages * Sh::kKVBytes / 16; i += 32)
-                        vr[i] = make_uint4(0u, 0u, 0u, 0u);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
                 // block ids of window w of a segment, lane l: entry w + l of the
                 // segment's block order (the prefix in table order; a member's
                 // last block first, then its blocks from 0)
@@ -500,8 +552,11 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                         // a member's partly filled last block is shifted to end at
                         // its slot's last row; the rows before it read as zero
                         const int shift = (wk.m >= 0 && kb0 + i == 0) ? wk.len - nb_seg * BS : 0;
-                        tma_load_4d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
-                                    bar(full0 + s), h * 64, kvh, shift, blk, policy);
+                        const uint32_t dst = ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128;
+                        if (shift)
+                            tma_load_4d(dst, tm4, bar(full0 + s), h * 64, kvh, shift, blk, policy);
+                        else
+                            tma_load_3d(dst, tm, bar(full0 + s), h * 64, kvh, blk * BS, policy);
                     }
                     issued = j + 1;
                     if (walk_next(wk)) {
@@ -513,76 +568,102 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                     }
                 }
             } else {
-            int ids = 0;
-            for (int j = 0; j < nt; ++j) {
-                const int s = j % NS;
-                if (j >= NS) {
-                    const bool free_ =
-                        mbar_wait_bounded(bar(empty0 + s), (uint32_t)((j / NS - 1) & 1), kWaitLimitNs);
-                    if (!__all_sync(0xffffffffu, free_)) {
-                        if (lane == 0)
-                            raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-                        break;
+            // work tiles in order; key tiles numbered across them (J) so the
+            // rings and their barriers carry over from one work tile to the next
+            Wk cur, nxt;
+            bool has_cur = next_work(cur);
+            bool has_nxt = has_cur && next_work(nxt);
+            // block ids, read 32 at a time (one per lane); the next work tile's
+            // first 32 are read while this one streams
+            int ids = has_cur && lane < cur.nblk ? __ldg(cur.trow + lane) : 0;
+            int ids_nxt = has_nxt && lane < nxt.nblk ? __ldg(nxt.trow + lane) : 0;
+            int J = 0;
+            bool ok = true;
+            while (has_cur && ok) {
+                for (int j = 0; j < cur.nt; ++j, ++J) {
+                    const int s = J % NS;
+                    if (J >= NS) {
+                        const bool free_ = mbar_wait_bounded(bar(empty0 + s), (uint32_t)((J / NS - 1) & 1),
+                                                             kWaitLimitNs);
+                        if (!__all_sync(0xffffffffu, free_)) {
+                            if (lane == 0)
+                                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+                            ok = false;
+                            break;
+                        }
                     }
-                }
-                const int kb0 = j * BPT;                   // a tile never straddles 32 ids
-                const int nb = min(BPT, nblk - kb0);
-                if ((kb0 & 31) == 0)
-                    ids = kb0 + lane < nblk ? __ldg(trow + kb0 + lane) : 0;
-                if (lane == 0)
-                    mbar_arrive_expect_tx(bar(full0 + s), (uint32_t)(nb * BS * D * 2));
-                __syncwarp();
-                // lane i * kHalves + h copies half h of the tile's block i: the
-                // tile's copies leave in one warp instruction, not one by one
-                const int i = lane / Sh::kHalves;
-                const int h = lane - i * Sh::kHalves;
-                int blk = __shfl_sync(0xffffffffu, ids, (kb0 + min(i, BPT - 1)) & 31);
-                if (i < nb) {
-                    if ((unsigned)blk >= (unsigned)num_blocks) {
-                        if (h == 0)
-                            raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
-                        blk = 0;
+                    const int kb0 = j * BPT;               // a tile never straddles 32 ids
+                    const int nb = min(BPT, cur.nblk - kb0);
+                    if (kb0 > 0 && (kb0 & 31) == 0)
+                        ids = kb0 + lane < cur.nblk ? __ldg(cur.trow + kb0 + lane) : 0;
+                    if (lane == 0)
+                        mbar_arrive_expect_tx(bar(full0 + s), (uint32_t)(nb * BS * D * 2));
+                    __syncwarp();
+                    // lane i * kHalves + h copies half h of the tile's block i: the
+                    // tile's copies leave in one warp instruction, not one by one
+                    const int i = lane / Sh::kHalves;
+                    const int h = lane - i * Sh::kHalves;
+                    int blk = __shfl_sync(0xffffffffu, ids, (kb0 + min(i, BPT - 1)) & 31);
+                    if (i < nb) {
+                        if ((unsigned)blk >= (unsigned)num_blocks) {
+                            if (h == 0)
+                                raise_flag(PKV_DEVFLAG_BLOCK_RANGE);
+                            blk = 0;
+                        }
+                        // the sequence's partly filled last block ends at its
+                        // slot's last row; the rows before it read as zero
+                        const int shift = (cur.tail && kb0 + i == cur.nblk - 1) ? cur.tail - BS : 0;
+                        const uint32_t dst = ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128;
+                        if (shift)
+                            tma_load_4d(dst, tm4, bar(full0 + s), h * 64, cur.kvh, shift, blk, policy);
+                        else
+                            tma_load_3d(dst, tm, bar(full0 + s), h * 64, cur.kvh, blk * BS, policy);
                     }
-                    tma_load_3d(ring + s * Sh::kKVBytes + h * Sh::kKVHalf + i * BS * 128, tm,
-                                bar(full0 + s), h * 64, kvh, blk * BS, policy);
+                    issued = J + 1;
                 }
-                issued = j + 1;
+                if (!ok)
+                    break;
+                cur = nxt;
+                has_cur = has_nxt;
+                ids = ids_nxt;
+                if (has_cur) {
+                    has_nxt = next_work(nxt);
+                    ids_nxt = has_nxt && lane < nxt.nblk ? __ldg(nxt.trow + lane) : 0;
+                }
             }
             }
-        }
-        if (MODE != kTcCascade && !is_k && issued == nt) {
-            // V rows of the last tile past p_max (the context's tail in its last
-            // block, and blocks never loaded) are cleared once the tile landed
-            const int j = nt - 1;
-            const int s = j % kPfVStages;
-            const bool landed =
-                mbar_wait_bounded(bar(kBarVFull + s), (uint32_t)((j / kPfVStages) & 1), kWaitLimitNs);
-            if (__all_sync(0xffffffffu, landed)) {
-                const int z0 = p_max + 1 - j * kPfKeys;   // first row to clear, 1 .. 64
-                if (z0 < kPfKeys) {
-                    uint8_t *vt = data + Sh::kVOff + s * Sh::kKVBytes;
-                    const int per_half = (kPfKeys - z0) * 8;   // 16-byte vectors
-                    for (int i = lane; i < Sh::kHalves * per_half; i += 32) {
-                        const int h = i / per_half;
-                        const int r = i - h * per_half;
-                        *reinterpret_cast<uint4 *>(vt + h * Sh::kKVHalf + (z0 + (r >> 3)) * 128 +
-                                                   (r & 7) * 16) = make_uint4(0u, 0u, 0u, 0u);
-                    }
-                }
-                fence_proxy_async_smem();
-            } else if (lane == 0) {
-                raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
-            }
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar(kBarVTail));
         }
         // copies still in flight land before the CTA can exit
         if (lane == 0) {
-            if (is_k)
-                mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs / 8);
             for (int j = issued > NS ? issued - NS : 0; j < issued; ++j)
                 mbar_wait_bounded(bar(full0 + j % NS), (uint32_t)((j / NS) & 1), kWaitLimitNs / 8);
+        }
+    } else if (warp == 7) {
+        // ---- Q of each work tile: the buffer is free once the previous work
+        // tile's last S = Q K^T has completed (the one-pass cascade holds its
+        // 32 rows four times) ----
+        if (lane == 0) {
+            constexpr int kCopies = MODE == kTcCascade ? 4 : 1;
+            const uint64_t policy = policy_evict_normal();
+            Wk wk;
+            int u = 0;
+            while (next_work(wk)) {
+                if (u > 0 && !mbar_wait_bounded(bar(kBarQEmpty), (uint32_t)((u - 1) & 1), kWaitLimitNs)) {
+                    raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+                    break;
+                }
+                mbar_arrive_expect_tx(bar(kBarQFull), (uint32_t)(kCopies * Sh::kHalves * R * 128));
+#pragma unroll
+                for (int q = 0; q < kCopies; ++q)
+#pragma unroll
+                    for (int h = 0; h < Sh::kHalves; ++h)
+                        tma_load_3d(sQ + h * Sh::kQHalf + q * 32 * 128, tm_q, bar(kBarQFull), h * 64,
+                                    wk.kvh * G, wk.q_tok0, policy);
+                ++u;
+            }
+            // the last Q lands before the CTA can exit
+            if (u > 0)
+                mbar_wait_bounded(bar(kBarQFull), (uint32_t)((u - 1) & 1), kWaitLimitNs / 8);
         }
     } else if (warp == 5) {
         // ---- MMA issue: one thread ----
@@ -612,37 +693,77 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 tc_commit(bar(kBarKEmpty + ks_));
                 return true;
             };
-            bool ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
-            for (int j = 0; ok && j < nt; ++j) {
-                if (j + 1 < nt) {
-                    // P_{j-1} V_{j-1} reads buffer (j+1) & 1.  O_DONE is at most
-                    // one phase past j-1 here: P_j V_j is not issued yet.
-                    if (j >= 1 &&
-                        !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs)))
+            // Key tiles are numbered across work tiles (J); S of the next key
+            // tile, in this work tile or the next, is issued before P V of the
+            // current one.  The last S of a work tile is followed by a commit to
+            // Q_EMPTY, which lets the loader bring the next work tile's Q.
+            Wk cur, nxt;
+            bool has_cur = next_work(cur);
+            bool has_nxt = has_cur && next_work(nxt);
+            bool ok = true;
+            if (has_cur) {
+                ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
+                if (ok && cur.nt == 1)
+                    tc_commit(bar(kBarQEmpty));
+            }
+            int J = 0;                              // the work tile's first key tile
+            int u = 0;                              // work tile index
+            while (ok && has_cur) {
+                for (int j = 0; ok && j < cur.nt; ++j) {
+                    const int Jj = J + j;
+                    const bool more = j + 1 < cur.nt;
+                    if (more) {
+                        // P_{Jj-1} V_{Jj-1} reads buffer (Jj+1) & 1.  O_DONE is at
+                        // most one phase past Jj-1 here: P_Jj V_Jj is not issued yet.
+                        if (Jj >= 1 &&
+                            !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((Jj - 1) & 1), kWaitLimitNs)))
+                            break;
+                        if (!(ok = issue_s(Jj + 1)))
+                            break;
+                        if (j + 2 == cur.nt)
+                            tc_commit(bar(kBarQEmpty));     // that S was the work tile's last
+                    }
+                    const int vs = Jj % kPfVStages;
+                    ok = mbar_wait_bounded(bar(kBarPFull + (Jj & 1)), (uint32_t)((Jj >> 1) & 1), kWaitLimitNs) &&
+                         mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((Jj / kPfVStages) & 1),
+                                           kWaitLimitNs);
+                    if (!ok)
                         break;
-                    if (!(ok = issue_s(j + 1)))
-                        break;
-                }
-                const int vs = j % kPfVStages;
-                ok = mbar_wait_bounded(bar(kBarPFull + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
-                     mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((j / kPfVStages) & 1),
-                                       kWaitLimitNs) &&
-                     (MODE == kTcCascade || j + 1 < nt ||
-                      mbar_wait_bounded(bar(kBarVTail), 0u, kWaitLimitNs));
-                if (!ok)
-                    break;
-                tc_fence_after();
-                // O += P_j V_j: P from TMEM (16 keys = 8 packed columns per
-                // k-step), V MN-major (head dim along the rows: halves LBO
-                // apart, 8-key groups 1024 bytes apart)
-                const uint32_t vt = sV + vs * Sh::kKVBytes;
-                const uint32_t tp = tmem + (j & 1) * kPfKeys;
+                    tc_fence_after();
+                    // O += P_j V_j: P from TMEM (16 keys = 8 packed columns per
+                    // k-step), V MN-major (head dim along the rows: halves LBO
+                    // apart, 8-key groups 1024 bytes apart); the work tile's first
+                    // P V overwrites O (its previous contents were read by the
+                    // softmax warps before they stored this P)
+                    const uint32_t vt = sV + vs * Sh::kKVBytes;
+                    const uint32_t tp = tmem + (Jj & 1) * kPfKeys;
 #pragma unroll
-                for (int kk = 0; kk < KV_STEPS; ++kk)
-                    tc_mma_f16_ts(tO, tp + kk * 8, sw128_desc(vt + kk * 16 * 128, Sh::kKVHalf, 1024),
-                                  idO, (j > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(bar(kBarODone));
-                tc_commit(bar(kBarVEmpty + vs));
+                    for (int kk = 0; kk < KV_STEPS; ++kk)
+                        tc_mma_f16_ts(tO, tp + kk * 8, sw128_desc(vt + kk * 16 * 128, Sh::kKVHalf, 1024),
+                                      idO, (j > 0 || kk > 0) ? 1u : 0u);
+                    tc_commit(bar(kBarODone));
+                    tc_commit(bar(kBarVEmpty + vs));
+                    if (!more && has_nxt) {
+                        // the next work tile's first S, after this work tile's
+                        // last P V (which must not wait for the next Q).  It
+                        // overwrites the buffer P_{Jj-1} V_{Jj-1} read: wait for
+                        // P_Jj V_Jj, which completes after it.  O_DONE is at most
+                        // one phase past Jj here: P_FULL of tile Jj came after
+                        // the softmax warps saw tile Jj-1's phase complete.
+                        if (!(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)(Jj & 1), kWaitLimitNs) &&
+                                   mbar_wait_bounded(bar(kBarQFull), (uint32_t)((u + 1) & 1), kWaitLimitNs) &&
+                                   issue_s(Jj + 1)))
+                            break;
+                        if (nxt.nt == 1)
+                            tc_commit(bar(kBarQEmpty));     // that S was its work tile's last
+                    }
+                }
+                J += cur.nt;
+                ++u;
+                cur = nxt;
+                has_cur = has_nxt;
+                if (has_cur)
+                    has_nxt = next_work(nxt);
             }
             if (!ok)
                 raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
@@ -831,21 +952,25 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         // ---- softmax and epilogue: thread = row r of the tile = TMEM lane r ----
         const int r = warp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const int grow = row0 + r;                  // row within the sequence
-        const bool real = r < R && grow < rows;
-        const int pos = real && MODE == kTcPrefill ? pos0 + r / G : p_max;
-        float m_used = kNegInf;
-        float l = 0.f;
-        bool ok = true;
         // for a positive scale the maximum is taken on the raw scores and the
         // scale is folded into the exponent, p = 2^(s*scale - m)
         const float sc = scale_log2;
         const bool fold = sc > 0.f;
         const float sm = fold ? 1.f : sc;       // applied before the maximum
         const float se = fold ? sc : 1.f;       // applied in the exponent
-        for (int j = 0; j < nt; ++j) {
-            const int s = j & 1;
-            ok = mbar_wait_bounded(bar(kBarSFull + s), (uint32_t)((j >> 1) & 1), kWaitLimitNs);
+        bool ok = true;
+        Wk cur;
+        int J = 0;                              // the work tile's first key tile
+        while (ok && next_work(cur)) {
+        const int grow = cur.row0 + r;          // row within the sequence
+        const bool real = r < R && grow < cur.rows;
+        const int pos = real && MODE == kTcPrefill ? cur.pos0 + r / G : cur.p_max;
+        float m_used = kNegInf;
+        float l = 0.f;
+        for (int j = 0; j < cur.nt; ++j) {
+            const int Jj = J + j;
+            const int s = Jj & 1;
+            ok = mbar_wait_bounded(bar(kBarSFull + s), (uint32_t)((Jj >> 1) & 1), kWaitLimitNs);
             if (!__all_sync(0xffffffffu, ok)) {
                 ok = false;
                 break;
@@ -860,17 +985,34 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             for (int i = 0; i < 8; ++i)
                 mx[i] = kNegInf;
             const int t0 = j * kPfKeys;
-            if (t0 + kPfKeys - 1 <= pos0) {         // every key visible to every row
+            if (t0 + kPfKeys - 1 <= cur.pos0) {     // every key visible to every row
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     x[c] = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
                     mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
-            } else {
+            } else if (!cur.tail || j + 1 < cur.nt) {   // causal mask, no shifted block
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const float v = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
                     x[c] = t0 + c <= pos ? v : kNegInf;
+                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+                }
+            } else {
+                // the work tile's last key tile holds the sequence's partly
+                // filled last block, loaded shifted: its slot starts with
+                // BS - tail rows of zeros (no key), then keys of positions
+                // t0 + c - (BS - tail); columns past it are past the context
+                const int sh_lo = (cur.nblk - 1 - j * BPT) * BS;
+                const int sh = BS - cur.tail;
+                const int nv = pos - t0 + 1;        // keys of this row in the tile, were none shifted
+                // visible columns: [0, min(nv, sh_lo)) and, in the shifted slot, [sh_lo + sh, nv + sh)
+                const uint64_t vm = col_range(0, min(nv, sh_lo)) | col_range(sh_lo + sh, nv + sh);
+                const uint32_t vlo = (uint32_t)vm, vhi = (uint32_t)(vm >> 32);
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    const float v = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
+                    x[c] = (((c < 32 ? vlo : vhi) >> (c & 31)) & 1u) ? v : kNegInf;
                     mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
             }
@@ -903,7 +1045,7 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 // no other.  O_DONE cannot be ahead of this wait either: P_j V_j
                 // needs this warp's P_j.  The MMA that may still run now is
                 // S_{j+1}, into the other S/P buffer.
-                ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs);
+                ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((Jj - 1) & 1), kWaitLimitNs);
                 if (!__all_sync(0xffffffffu, ok)) {
                     ok = false;
                     break;
@@ -930,12 +1072,14 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 mbar_arrive(bar(kBarPFull + s));
         }
         if (ok)
-            ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((nt - 1) & 1), kWaitLimitNs);
-        if (__all_sync(0xffffffffu, ok)) {
+            ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((J + cur.nt - 1) & 1), kWaitLimitNs);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
             tc_fence_after();
             const float inv = l > 0.f ? 1.f / l : 0.f;
             // query row (q_tok0 + r / G, head kvh * G + r % G): row0 is a multiple of G
-            const size_t orow_i = (size_t)(q_tok0 + r / G) * num_heads + (size_t)kvh * G + r % G;
+            const size_t orow_i =
+                (size_t)(cur.q_tok0 + r / G) * num_heads + (size_t)cur.kvh * G + r % G;
             if constexpr (MODE == kTcPrefill) {
                 uint4 *orow = reinterpret_cast<uint4 *>(a.out + orow_i * D);
 #pragma unroll 1
@@ -976,9 +1120,13 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                     c.rec_l[rec] = l;
                 }
             }
-        } else if (lane == 0) {
-            raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
+            // the next work tile's first P V overwrites O: these reads of O
+            // complete (tcgen05.wait::ld) before this warp stores that tile's P
         }
+        J += cur.nt;
+        }
+        if (!ok && lane == 0)
+            raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
     }
 
     // ---- release the tensor memory once every warp is done with it ----
@@ -991,31 +1139,36 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
     }
 }
 
+// tm_k / tm_v view the caches as 3-D tensors {head_dim, num_kv_heads,
+// num_blocks * block_size} (box 64 x 1 x block_size), tm_k4 / tm_v4 as 4-D
+// tensors {head_dim, num_kv_heads, block_size, num_blocks} (box 64 x 1 x
+// block_size x 1): whole blocks come through the first, a partly filled last
+// block, shifted so that the rows before it read as zero, through the second.
 template <int D, int BS, bool BF16>
 __global__ void __launch_bounds__(kPfThreads, 2)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const PrefillArgs a)
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k4,
+                  const __grid_constant__ CUtensorMap tm_v4, const PrefillArgs a)
 {
-    tc_attend<D, BS, BF16, kTcPrefill>(&tm_q, &tm_k, &tm_v, a, CascadeArgs{});
+    tc_attend<D, BS, BF16, kTcPrefill>(&tm_q, &tm_k, &tm_v, &tm_k4, &tm_v4, a, CascadeArgs{});
 }
 
 template <int D, int BS, bool BF16>
 __global__ void __launch_bounds__(kPfThreads, 2)
 prefix_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                 const __grid_constant__ CUtensorMap tm_v, const CascadeArgs c)
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k4,
+                 const __grid_constant__ CUtensorMap tm_v4, const CascadeArgs c)
 {
-    tc_attend<D, BS, BF16, kTcPrefix>(&tm_q, &tm_k, &tm_v, PrefillArgs{}, c);
+    tc_attend<D, BS, BF16, kTcPrefix>(&tm_q, &tm_k, &tm_v, &tm_k4, &tm_v4, PrefillArgs{}, c);
 }
 
-// One-pass cascade decode: tm_k / tm_v view the caches as 4-D tensors
-// {head_dim, num_kv_heads, block_size, num_blocks} (box 64 x 1 x block_size
-// x 1), so that a shifted load of a partly filled block reads zeros before it.
 template <int D, int BS, bool BF16>
 __global__ void __launch_bounds__(kPfThreads, 2)
 cascade_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const CascadeArgs c)
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k4,
+                  const __grid_constant__ CUtensorMap tm_v4, const CascadeArgs c)
 {
-    tc_attend<D, BS, BF16, kTcCascade>(&tm_q, &tm_k, &tm_v, PrefillArgs{}, c);
+    tc_attend<D, BS, BF16, kTcCascade>(&tm_q, &tm_k, &tm_v, &tm_k4, &tm_v4, PrefillArgs{}, c);
 }
 
 }  // namespace pkv

@@ -93,3 +93,44 @@ def test_prefill_growing_scores(dtype, D):
     step["value_cache"] = (step["value_cache"].float() * 0.25).to(_DT[dtype])
     q = (q.float() * 2.0).to(_DT[dtype])
     _check(step, q, qs, chunks)
+
+
+@pytest.mark.parametrize("bs", [16, 32])
+def test_prefill_garbage_past_the_context(bs):
+    """Cells past each sequence's last token (in its last block) hold NaN and
+    infinity: they are never read as keys or values, so every output stays
+    finite and within tolerance.  Lengths end inside a block, on a block
+    edge, and inside a 64-key tile."""
+    lens = [520, 7, 64, 65, 300, 17, 128, 33]
+    chunks = [7, 7, 64, 1, 300, 9, 5, 33]
+    step, q, qs = _case(lens, chunks, 8, 2, 128, bs, "bf16", seed=bs + 11)
+    kc, vc = step["key_cache"].clone(), step["value_cache"].clone()
+    for s_, L in enumerate(lens):
+        if L % bs:
+            blk = int(step["block_tables"][s_, (L - 1) // bs])
+            kc[blk, L % bs:] = float("nan")
+            vc[blk, L % bs:] = float("inf")
+    ref = oracle.paged_attention_prefill(u16(q), qs.numpy(), u16(step["key_cache"]),
+                                         u16(step["value_cache"]), step["block_tables"].numpy(),
+                                         step["context_lens"].numpy(), step["scale"], "bf16",
+                                         nthreads=NTHREADS)
+    d = {k: (v.cuda() if isinstance(v, torch.Tensor) else v) for k, v in step.items()}
+    out = pkv.paged_attention_prefill(q.cuda(), qs.cuda(), max(chunks), kc.cuda(), vc.cuda(),
+                                      d["block_tables"], d["context_lens"], step["scale"])
+    err, idx, finite = max_abs_err(out, ref)
+    assert finite and err <= TOL["bf16"], (err, idx)
+
+
+def test_prefill_many_work_tiles_per_cta():
+    """More row tiles than two per SM: the persistent CTAs walk several work
+    tiles each, of very different lengths (chunks of 1 to 1000 tokens).
+    Chunks that start a context give outputs over one or two keys, i.e. single
+    V entries; among 79M outputs some exceed 4 in magnitude, where rounding to
+    bf16 alone can pass the fixed absolute bound.  V is halved so that outputs
+    stay below 4, where the bound covers the final rounding."""
+    rng = np.random.default_rng(12)
+    lens = [int(x) for x in rng.integers(1, 1100, size=96)]
+    chunks = [int(min(L, c)) for L, c in zip(lens, rng.integers(1, 1000, size=96))]
+    step, q, qs = _case(lens, chunks, 16, 4, 128, 16, "bf16", seed=13)
+    step["value_cache"] = (step["value_cache"].float() * 0.5).to(torch.bfloat16)
+    _check(step, q, qs, chunks)
