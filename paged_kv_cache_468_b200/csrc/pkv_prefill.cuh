@@ -693,77 +693,109 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 tc_commit(bar(kBarKEmpty + ks_));
                 return true;
             };
-            // Key tiles are numbered across work tiles (J); S of the next key
-            // tile, in this work tile or the next, is issued before P V of the
-            // current one.  The last S of a work tile is followed by a commit to
-            // Q_EMPTY, which lets the loader bring the next work tile's Q.
-            Wk cur, nxt;
-            bool has_cur = next_work(cur);
-            bool has_nxt = has_cur && next_work(nxt);
             bool ok = true;
-            if (has_cur) {
+            if constexpr (MODE != kTcPrefill) {
+                // One work tile (the prefix pass and the one-pass cascade).  This
+                // plain loop is kept apart from the prefill's loop over several
+                // work tiles below: running the one-pass cascade through that
+                // loop made it 5 % slower.
                 ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
-                if (ok && cur.nt == 1)
-                    tc_commit(bar(kBarQEmpty));
-            }
-            int J = 0;                              // the work tile's first key tile
-            int u = 0;                              // work tile index
-            while (ok && has_cur) {
-                for (int j = 0; ok && j < cur.nt; ++j) {
-                    const int Jj = J + j;
-                    const bool more = j + 1 < cur.nt;
-                    if (more) {
-                        // P_{Jj-1} V_{Jj-1} reads buffer (Jj+1) & 1.  O_DONE is at
-                        // most one phase past Jj-1 here: P_Jj V_Jj is not issued yet.
-                        if (Jj >= 1 &&
-                            !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((Jj - 1) & 1), kWaitLimitNs)))
+                for (int j = 0; ok && j < nt; ++j) {
+                    if (j + 1 < nt) {
+                        // P_{j-1} V_{j-1} reads buffer (j+1) & 1.  O_DONE is at most
+                        // one phase past j-1 here: P_j V_j is not issued yet.
+                        if (j >= 1 &&
+                            !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((j - 1) & 1), kWaitLimitNs)))
                             break;
-                        if (!(ok = issue_s(Jj + 1)))
+                        if (!(ok = issue_s(j + 1)))
                             break;
-                        if (j + 2 == cur.nt)
-                            tc_commit(bar(kBarQEmpty));     // that S was the work tile's last
                     }
-                    const int vs = Jj % kPfVStages;
-                    ok = mbar_wait_bounded(bar(kBarPFull + (Jj & 1)), (uint32_t)((Jj >> 1) & 1), kWaitLimitNs) &&
-                         mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((Jj / kPfVStages) & 1),
+                    const int vs = j % kPfVStages;
+                    ok = mbar_wait_bounded(bar(kBarPFull + (j & 1)), (uint32_t)((j >> 1) & 1), kWaitLimitNs) &&
+                         mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((j / kPfVStages) & 1),
                                            kWaitLimitNs);
                     if (!ok)
                         break;
                     tc_fence_after();
-                    // O += P_j V_j: P from TMEM (16 keys = 8 packed columns per
-                    // k-step), V MN-major (head dim along the rows: halves LBO
-                    // apart, 8-key groups 1024 bytes apart); the work tile's first
-                    // P V overwrites O (its previous contents were read by the
-                    // softmax warps before they stored this P)
+                    // O += P_j V_j, as below
                     const uint32_t vt = sV + vs * Sh::kKVBytes;
-                    const uint32_t tp = tmem + (Jj & 1) * kPfKeys;
+                    const uint32_t tp = tmem + (j & 1) * kPfKeys;
 #pragma unroll
                     for (int kk = 0; kk < KV_STEPS; ++kk)
                         tc_mma_f16_ts(tO, tp + kk * 8, sw128_desc(vt + kk * 16 * 128, Sh::kKVHalf, 1024),
                                       idO, (j > 0 || kk > 0) ? 1u : 0u);
                     tc_commit(bar(kBarODone));
                     tc_commit(bar(kBarVEmpty + vs));
-                    if (!more && has_nxt) {
+                }
+            } else {
+                // Key tiles are numbered across the CTA's work tiles (J), in one
+                // loop; the current work tile holds key tiles Jbeg .. Jend-1.  S
+                // of the next key tile, in this work tile or the next, is issued
+                // before P V of the current one.  The last S of a work tile is
+                // followed by a commit to Q_EMPTY, which lets the loader bring the
+                // next work tile's Q.
+                Wk nxt;
+                int Jend = 0;
+                bool has_nxt = false;
+                if (next_work(nxt)) {
+                    Jend = nxt.nt;
+                    has_nxt = next_work(nxt);
+                    ok = mbar_wait_bounded(bar(kBarQFull), 0u, kWaitLimitNs) && issue_s(0);
+                    if (ok && Jend == 1)
+                        tc_commit(bar(kBarQEmpty));
+                }
+                int Jbeg = 0;
+                int u = 0;                              // work tile index
+                for (int J = 0; ok && J < Jend; ++J) {
+                    if (J + 1 < Jend) {
+                        // P_{J-1} V_{J-1} reads buffer (J+1) & 1.  O_DONE is at most
+                        // one phase past J-1 here: P_J V_J is not issued yet.
+                        if (J >= 1 &&
+                            !(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)((J - 1) & 1), kWaitLimitNs)))
+                            break;
+                        if (!(ok = issue_s(J + 1)))
+                            break;
+                        if (J + 2 == Jend)
+                            tc_commit(bar(kBarQEmpty));         // that S was the work tile's last
+                    }
+                    const int vs = J % kPfVStages;
+                    ok = mbar_wait_bounded(bar(kBarPFull + (J & 1)), (uint32_t)((J >> 1) & 1), kWaitLimitNs) &&
+                         mbar_wait_bounded(bar(kBarVFull + vs), (uint32_t)((J / kPfVStages) & 1), kWaitLimitNs);
+                    if (!ok)
+                        break;
+                    tc_fence_after();
+                    // O += P_J V_J: P from TMEM (16 keys = 8 packed columns per
+                    // k-step), V MN-major (head dim along the rows: halves LBO
+                    // apart, 8-key groups 1024 bytes apart); the work tile's first
+                    // P V overwrites O (its previous contents were read by the
+                    // softmax warps before they stored this P)
+                    const uint32_t vt = sV + vs * Sh::kKVBytes;
+                    const uint32_t tp = tmem + (J & 1) * kPfKeys;
+#pragma unroll
+                    for (int kk = 0; kk < KV_STEPS; ++kk)
+                        tc_mma_f16_ts(tO, tp + kk * 8, sw128_desc(vt + kk * 16 * 128, Sh::kKVHalf, 1024),
+                                      idO, (J > Jbeg || kk > 0) ? 1u : 0u);
+                    tc_commit(bar(kBarODone));
+                    tc_commit(bar(kBarVEmpty + vs));
+                    if (J + 1 == Jend && has_nxt) {
                         // the next work tile's first S, after this work tile's
                         // last P V (which must not wait for the next Q).  It
-                        // overwrites the buffer P_{Jj-1} V_{Jj-1} read: wait for
-                        // P_Jj V_Jj, which completes after it.  O_DONE is at most
-                        // one phase past Jj here: P_FULL of tile Jj came after
-                        // the softmax warps saw tile Jj-1's phase complete.
-                        if (!(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)(Jj & 1), kWaitLimitNs) &&
+                        // overwrites the buffer P_{J-1} V_{J-1} read: wait for
+                        // P_J V_J, which completes after it.  O_DONE is at most
+                        // one phase past J here: P_FULL of tile J came after the
+                        // softmax warps saw tile J-1's phase complete.
+                        if (!(ok = mbar_wait_bounded(bar(kBarODone), (uint32_t)(J & 1), kWaitLimitNs) &&
                                    mbar_wait_bounded(bar(kBarQFull), (uint32_t)((u + 1) & 1), kWaitLimitNs) &&
-                                   issue_s(Jj + 1)))
+                                   issue_s(J + 1)))
                             break;
+                        ++u;
+                        Jbeg = J + 1;
+                        Jend += nxt.nt;
                         if (nxt.nt == 1)
-                            tc_commit(bar(kBarQEmpty));     // that S was its work tile's last
+                            tc_commit(bar(kBarQEmpty));         // that S was its work tile's last
+                        has_nxt = next_work(nxt);
                     }
                 }
-                J += cur.nt;
-                ++u;
-                cur = nxt;
-                has_cur = has_nxt;
-                if (has_cur)
-                    has_nxt = next_work(nxt);
             }
             if (!ok)
                 raise_flag(PKV_DEVFLAG_WAIT_TIMEOUT);
@@ -978,25 +1010,18 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             tc_fence_after();
             uint32_t raw[64];
             tmem_ld64(tmem + lane_base + s * kPfKeys, raw);
-            // eight independent max / sum chains, not 64-long ones
+            // the scores with the mask applied (-inf where a row sees no key)
             float x[64];
-            float mx[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                mx[i] = kNegInf;
             const int t0 = j * kPfKeys;
             if (t0 + kPfKeys - 1 <= cur.pos0) {     // every key visible to every row
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
+                for (int c = 0; c < 64; ++c)
                     x[c] = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
-                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-                }
             } else if (!cur.tail || j + 1 < cur.nt) {   // causal mask, no shifted block
 #pragma unroll
                 for (int c = 0; c < 64; ++c) {
                     const float v = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
                     x[c] = t0 + c <= pos ? v : kNegInf;
-                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
             } else {
                 // the work tile's last key tile holds the sequence's partly
@@ -1013,29 +1038,36 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
                 for (int c = 0; c < 64; ++c) {
                     const float v = fold ? __uint_as_float(raw[c]) : __uint_as_float(raw[c]) * sm;
                     x[c] = (((c < 32 ? vlo : vhi) >> (c & 31)) & 1u) ? v : kNegInf;
-                    mx[c & 7] = fmaxf(mx[c & 7], x[c]);
                 }
             }
-            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * se;
+            // eight independent max chains of three-input maxima, not a 64-long one
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                mx[i] = fmaxf(x[2 * i], x[2 * i + 1]);
+#pragma unroll
+            for (int c = 16; c < 64; c += 2)
+                mx[(c >> 1) & 7] = fmax3(mx[(c >> 1) & 7], x[c], x[c + 1]);
+            const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * se;
             const bool resc = mt > m_used + 8.f;    // first tile: m_used = -inf
             const float m_new = resc ? mt : m_used;
             const float alpha = resc ? ex2(m_used - m_new) : 1.f;
             const float msub = m_new == kNegInf ? 0.f : m_new;
-            // the row sum is taken over the rounded weights the MMA multiplies,
-            // so the normalised weights sum to one exactly
+            // exponents two columns at a time (packed f32x2 fma); the row sum is
+            // taken over the rounded weights the MMA multiplies, so the
+            // normalised weights sum to one exactly (four packed chains)
+            const uint64_t se2 = f2(se, se), nm2 = f2(-msub, -msub);
             uint32_t pk[32];
-            float rsv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                rsv[i] = 0.f;
+            uint64_t rsv[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                pk[c] = pack2<BF16>(ex2(fmaf(x[2 * c], se, -msub)), ex2(fmaf(x[2 * c + 1], se, -msub)));
+                const uint64_t e = fma2(f2(x[2 * c], x[2 * c + 1]), se2, nm2);
+                pk[c] = pack2<BF16>(ex2(f2_lo(e)), ex2(f2_hi(e)));
                 const float2 pr = unpack2<BF16>(pk[c]);
-                rsv[c & 7] += pr.x + pr.y;
+                rsv[c & 3] = add2(rsv[c & 3], f2(pr.x, pr.y));
             }
-            const float rs = ((rsv[0] + rsv[1]) + (rsv[2] + rsv[3])) + ((rsv[4] + rsv[5]) + (rsv[6] + rsv[7]));
+            const uint64_t r2 = add2(add2(rsv[0], rsv[1]), add2(rsv[2], rsv[3]));
+            const float rs = f2_lo(r2) + f2_hi(r2);
             l = l * alpha + rs;
             m_used = m_new;
             if (j > 0) {

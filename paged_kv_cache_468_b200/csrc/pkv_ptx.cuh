@@ -2,7 +2,8 @@
 //
 // Only documented PTX instructions appear here (mbarrier, cp.async.bulk.tensor
 // without multicast, ldmatrix, mma.sync m16n8k16, movmatrix, ex2.approx,
-// tcgen05 alloc / mma / commit / ld / st).
+// packed f32x2 add / fma, three-input max, tcgen05 alloc / mma / commit /
+// ld / st).
 #pragma once
 
 #include <cstdint>
@@ -171,6 +172,38 @@ __device__ __forceinline__ float ex2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// ---- sm_100 packed FP32: two f32 lanes in a 64-bit register pair ----
+__device__ __forceinline__ uint64_t f2(float lo, float hi)
+{
+    return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+// a * b + c, lane by lane, each lane rounded as one fma.rn.f32
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+// a + b, lane by lane
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // ---- tcgen05: 5th-generation tensor cores, accumulators in tensor memory ----
