@@ -551,9 +551,12 @@ def measure_decode_launches(w: DecodeWorkload, n: int, stream, flush_buf, sample
             "p90_ms": q[-1], "n": n, "timing": timing}
 
 
-def read_ceiling(pkv, dev, stream, nbytes: int = 2 << 30, reps: int = 40) -> dict:
+def read_ceiling(pkv, dev, stream, nbytes: int = 2 << 30, reps: int = 40, same_bytes: int = 0) -> dict:
     """Read-only HBM streaming rate (16-byte loads over nbytes), best over a
-    few grid sizes: the ceiling of a kernel that only reads."""
+    few grid sizes: the ceiling of a kernel that only reads.  With same_bytes,
+    also the rate of reading just that many bytes (the decode call's) as
+    scattered 4 KiB chunks, launched back to back like the decode: a short
+    kernel pays its ramp-up and drain too."""
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     buf = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     buf.fill_(1)
@@ -580,11 +583,31 @@ def read_ceiling(pkv, dev, stream, nbytes: int = 2 << 30, reps: int = 40) -> dic
             fn()
         ms = time_back_to_back(fn, reps, stream)
         gather[str(grid)] = round(nbytes / (ms * 1e-3) / 1e9, 1)
+    same = {}
+    n_same = min(-(-same_bytes // chunk), nbytes // chunk)
+    if n_same > 0:
+        # the first n_same chunks of the buffer (a pool the size of the decode's
+        # blocks), each read once, in a random order
+        buf_s = buf[:n_same * chunk]
+        order_s = torch.randperm(n_same, generator=torch.Generator().manual_seed(6)).to(torch.int32).to(dev)
+        launches = max(reps, int(0.3 / (n_same * chunk / 7e12)))    # ~0.3 s at 7 TB/s
+        for per_sm in (2, 4, 8):
+            grid = sms * per_sm
+            fn = lambda: pkv.hbm_gather_probe(buf_s, chunk, order_s, sink, grid)
+            for _ in range(3):
+                fn()
+            ms = time_back_to_back(fn, launches, stream)
+            same[str(grid)] = round(n_same * chunk / (ms * 1e-3) / 1e9, 1)
+        del order_s, buf_s
     del buf, order
-    return {"gbs": max(rates.values()), "bytes": nbytes, "reps": reps, "by_grid": rates,
-            "kernel": "hbm_read_probe_kernel (16-byte ld.global.nc, 8 in flight per thread)",
-            "gather_4k_gbs": max(gather.values()), "gather_4k_by_grid": gather,
-            "gather_kernel": "hbm_gather_probe_kernel (4 KiB chunks in a random order, a warp per chunk)"}
+    r = {"gbs": max(rates.values()), "bytes": nbytes, "reps": reps, "by_grid": rates,
+         "kernel": "hbm_read_probe_kernel (16-byte ld.global.nc, 8 in flight per thread)",
+         "gather_4k_gbs": max(gather.values()), "gather_4k_by_grid": gather,
+         "gather_kernel": "hbm_gather_probe_kernel (4 KiB chunks in a random order, a warp per chunk)"}
+    if same:
+        r.update({"same_size_gather_gbs": max(same.values()), "same_size_bytes": n_same * chunk,
+                  "same_size_by_grid": same, "same_size_launches": launches})
+    return r
 
 
 def roofline_entry(w: DecodeWorkload, t: dict, peaks: dict, ceiling) -> dict:
@@ -605,6 +628,9 @@ def roofline_entry(w: DecodeWorkload, t: dict, peaks: dict, ceiling) -> dict:
         r["frac_of_read_ceiling"] = round(achieved / ceiling["gbs"], 4)
         r["gather_ceiling_gbs"] = ceiling["gather_4k_gbs"]
         r["frac_of_gather_ceiling"] = round(achieved / ceiling["gather_4k_gbs"], 4)
+        if "same_size_gather_gbs" in ceiling and abs(ceiling["same_size_bytes"] - bytes_) <= 0.1 * bytes_:
+            r["same_size_gather_gbs"] = ceiling["same_size_gather_gbs"]
+            r["frac_of_same_size_gather"] = round(achieved / ceiling["same_size_gather_gbs"], 4)
     return r
 
 
@@ -786,7 +812,7 @@ def run_gpu(args, cfg, world, rank, local):
     per_config = None
     if rank == 0 and world == 1:
         if not args.no_read_ceiling:
-            ceiling = read_ceiling(pkv, dev, stream)
+            ceiling = read_ceiling(pkv, dev, stream, same_bytes=nbytes["decode_unique"])
         if not args.no_per_config:
             per_config = {}
             for name in workloads.CONFIGS:

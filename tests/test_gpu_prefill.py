@@ -100,9 +100,9 @@ def test_prefill_garbage_past_the_context(bs):
     """Cells past each sequence's last token (in its last block) hold NaN and
     infinity: they are never read as keys or values, so every output stays
     finite and within tolerance.  Lengths end inside a block, on a block
-    edge, and inside a 64-key tile."""
-    lens = [520, 7, 64, 65, 300, 17, 128, 33]
-    chunks = [7, 7, 64, 1, 300, 9, 5, 33]
+    edge, on a key-tile edge and inside a key tile."""
+    lens = [520, 7, 64, 65, 300, 17, 128, 33, 129, 255, 256, 257]
+    chunks = [7, 7, 64, 1, 300, 9, 5, 33, 129, 100, 3, 257]
     step, q, qs = _case(lens, chunks, 8, 2, 128, bs, "bf16", seed=bs + 11)
     kc, vc = step["key_cache"].clone(), step["value_cache"].clone()
     for s_, L in enumerate(lens):
