@@ -198,13 +198,17 @@ __device__ __forceinline__ void attend_block(uint32_t sk, uint32_t sv, int valid
         mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 8));
         mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], 16));
     }
+    // The running maximum moves only when a block's maximum exceeds it by
+    // more than 8 (base 2), so the weights stay <= 2^8 and O and the
+    // normaliser are rescaled only then, not on every block that raises the
+    // maximum a little.  alpha is 0 on a column's first scored block
+    // (m_run = -inf) and 1 while a column has seen no token at all.
     float alpha[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        const float mnew = fmaxf(m_run[j], mx[j]);
-        // 0 on a column's first scored block (m_run = -inf); 1 while a column
-        // has seen no token at all (both -inf)
-        alpha[j] = mnew == kNegInf ? 1.f : ex2(m_run[j] - mnew);
+        const bool move = mx[j] > m_run[j] + 8.f;
+        const float mnew = move ? mx[j] : m_run[j];
+        alpha[j] = move ? ex2(m_run[j] - mnew) : 1.f;
         m_run[j] = mnew;
     }
     float ls[2] = {0.f, 0.f};
@@ -219,16 +223,18 @@ __device__ __forceinline__ void attend_block(uint32_t sk, uint32_t sv, int valid
 #pragma unroll
     for (int j = 0; j < 2; ++j)
         l_run[j] = l_run[j] * alpha[j] + ls[j];
+    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-    for (int dt = 0; dt < KS; ++dt) {
-        acc_hi[dt][0] *= alpha[0];
-        acc_hi[dt][1] *= alpha[1];
-        acc_hi[dt][2] *= alpha[0];
-        acc_hi[dt][3] *= alpha[1];
-        acc_lo[dt][0] *= alpha[0];
-        acc_lo[dt][1] *= alpha[1];
-        acc_lo[dt][2] *= alpha[0];
-        acc_lo[dt][3] *= alpha[1];
+        for (int dt = 0; dt < KS; ++dt) {
+            acc_hi[dt][0] *= alpha[0];
+            acc_hi[dt][1] *= alpha[1];
+            acc_hi[dt][2] *= alpha[0];
+            acc_hi[dt][3] *= alpha[1];
+            acc_lo[dt][0] *= alpha[0];
+            acc_lo[dt][1] *= alpha[1];
+            acc_lo[dt][2] *= alpha[0];
+            acc_lo[dt][3] *= alpha[1];
+        }
     }
 
     // ---- O^T[d, n] += sum_t V[t, d] P[t, n] ----
