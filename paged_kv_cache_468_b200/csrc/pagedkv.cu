@@ -186,7 +186,7 @@ struct Tuning { static constexpr int NW = PKV_TUNE_NW, S = PKV_TUNE_S; };
 template <> struct Tuning<64, 16>  { static constexpr int NW = 4, S = 2; };   // 33 KB, 6 CTAs/SM
 template <> struct Tuning<64, 32>  { static constexpr int NW = 2, S = 3; };   // 49 KB
 template <> struct Tuning<128, 16> { static constexpr int NW = 2, S = 2; };   // 33 KB, 6 CTAs/SM
-template <> struct Tuning<128, 32> { static constexpr int NW = 2, S = 3; };   // 97 KB, 2 CTAs/SM
+template <> struct Tuning<128, 32> { static constexpr int NW = 2, S = 2; };   // 65 KB, 3 CTAs/SM
 #endif
 
 int current_device()
