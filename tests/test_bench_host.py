@@ -54,3 +54,24 @@ def test_committed_traffic_entries_are_well_formed():
         if name == "note":
             continue
         assert entry["dram_bytes_per_launch"] > 0 and len(entry["source_sha"]) == 16
+
+
+def test_packed_inputs_round_trip_at_aligned_offsets():
+    """The end-to-end step uploads its inputs as one packed buffer: every
+    tensor sits at a 256-byte aligned offset and reads back unchanged through
+    its view, after a byte copy of the whole buffer."""
+    import torch
+    src = {"query": torch.randn(3, 4, 8).to(torch.bfloat16),
+           "slot_mapping": torch.arange(5, dtype=torch.int64) * 7,
+           "block_tables": torch.arange(12, dtype=torch.int32).view(3, 4),
+           "context_lens": torch.tensor([1, 2, 3], dtype=torch.int32)}
+    hbuf, hview = bench._packed(src, lambda n: torch.zeros(n, dtype=torch.uint8))
+    for k, v in src.items():
+        hview[k].copy_(v)
+    dbuf, dview = bench._packed(src, lambda n: torch.full((n,), 255, dtype=torch.uint8))
+    dbuf.copy_(hbuf)
+    for k, v in src.items():
+        assert dview[k].shape == v.shape and dview[k].dtype == v.dtype
+        assert (dview[k].storage_offset() * dview[k].element_size()) % 256 == 0
+        assert torch.equal(dview[k], v), k
+    assert hbuf.numel() % 256 == 0
