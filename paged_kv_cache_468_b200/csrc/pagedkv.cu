@@ -449,11 +449,10 @@ pkv_status pkv_kv_cache_write(const void *key, const void *value, const int64_t 
     if (blocks > 148 * 16)
         blocks = 148 * 16;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    pkv::kv_write_kernel<<<(unsigned)blocks, threads, 0, st>>>(
-        static_cast<const uint4 *>(key), static_cast<const uint4 *>(value), slot_mapping, n_vec,
-        vec_per_token, num_blocks * block_size, static_cast<uint4 *>(key_cache),
-        static_cast<uint4 *>(value_cache));
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(pkv::kv_write_kernel, dim3((unsigned)blocks), dim3(threads), 0, st,
+                               static_cast<const uint4 *>(key), static_cast<const uint4 *>(value),
+                               slot_mapping, n_vec, vec_per_token, num_blocks * block_size,
+                               static_cast<uint4 *>(key_cache), static_cast<uint4 *>(value_cache));
     if (e != cudaSuccess)
         return cuda_fail(e, "kv_write_kernel launch");
     return PKV_OK;

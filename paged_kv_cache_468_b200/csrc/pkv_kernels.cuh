@@ -111,8 +111,13 @@ __global__ void kv_write_kernel(const uint4 *__restrict__ key, const uint4 *__re
                                 int64_t vec_per_token, int64_t total_slots,
                                 uint4 *__restrict__ key_cache, uint4 *__restrict__ value_cache)
 {
-    // A decode launched after this kernel may start its own set-up now; it
-    // waits for this grid to finish before it reads any memory.
+    // Launched with programmatic dependent launch, this grid may become
+    // resident while the previous kernel on the stream finishes (its launch
+    // latency is then hidden): it waits for that kernel before it touches
+    // memory, which may have read these cells or written these inputs.  A
+    // decode launched after this kernel may start its own set-up now; it waits
+    // for this grid to finish before it reads any memory.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n_vec; i += stride) {
