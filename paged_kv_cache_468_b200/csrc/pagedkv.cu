@@ -399,11 +399,11 @@ pkv_status pkv_copy_blocks(const void *src_key_cache, const void *src_value_cach
         return fail(PKV_ERR_MISALIGNED, "block_mapping must be 8-byte aligned");
     const int64_t vec_per_block = block_bytes / 16;
     const int64_t blocks = 2 * (int64_t)num_pairs;   // one CTA per (pair, K or V)
-    pkv::copy_blocks_kernel<<<(unsigned)blocks, pkv::kCopyThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4 *>(src_key_cache), static_cast<const uint4 *>(src_value_cache),
-        static_cast<uint4 *>(dst_key_cache), static_cast<uint4 *>(dst_value_cache), block_mapping,
-        num_pairs, src_num_blocks, dst_num_blocks, vec_per_block);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(pkv::copy_blocks_kernel, dim3((unsigned)blocks), dim3(pkv::kCopyThreads), 0,
+                               static_cast<cudaStream_t>(stream),
+                               static_cast<const uint4 *>(src_key_cache), static_cast<const uint4 *>(src_value_cache),
+                               static_cast<uint4 *>(dst_key_cache), static_cast<uint4 *>(dst_value_cache),
+                               block_mapping, num_pairs, src_num_blocks, dst_num_blocks, vec_per_block);
     if (e != cudaSuccess)
         return cuda_fail(e, "copy_blocks_kernel launch");
     return PKV_OK;

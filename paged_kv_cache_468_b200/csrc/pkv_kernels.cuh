@@ -730,6 +730,10 @@ copy_blocks_kernel(const uint4 *__restrict__ src_k, const uint4 *__restrict__ sr
                    const int32_t *__restrict__ mapping, int num_pairs, int64_t src_blocks,
                    int64_t dst_blocks, int64_t vec_per_block)
 {
+    // Launched with programmatic dependent launch: wait for the previous
+    // kernel on the stream before touching memory, then let the next start.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int64_t pair = blockIdx.x >> 1;
     const bool is_v = blockIdx.x & 1;
     if (pair >= num_pairs)

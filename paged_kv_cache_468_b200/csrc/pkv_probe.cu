@@ -32,9 +32,29 @@ __device__ __forceinline__ uint4 load_stream(const uint4 *p)
     return v;
 }
 
+// Launched like the decode kernels (programmatic dependent launch), so that
+// back-to-back launches overlap one launch's start with the previous one's
+// end exactly as the decode's do.
+template <typename Kernel, typename... Args>
+cudaError_t launch_pdl(Kernel kern, unsigned grid, void *stream, Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kProbeThreads);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 __global__ void __launch_bounds__(kProbeThreads)
 hbm_read_probe_kernel(const uint4 *__restrict__ buf, int64_t n_vec, uint32_t *__restrict__ sink)
 {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int64_t stride = (int64_t)gridDim.x * kProbeThreads;
     int64_t i = (int64_t)blockIdx.x * kProbeThreads + threadIdx.x;
     uint32_t acc = 0;
@@ -66,6 +86,8 @@ __global__ void __launch_bounds__(kProbeThreads)
 hbm_gather_probe_kernel(const uint4 *__restrict__ buf, const int32_t *__restrict__ order,
                         int64_t n_chunks, int64_t vec_per_chunk, uint32_t *__restrict__ sink)
 {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int lane = threadIdx.x & 31;
     const int64_t nw = (int64_t)gridDim.x * (kProbeThreads / 32);
     uint32_t acc = 0;
@@ -105,9 +127,8 @@ extern "C" pkv_status pkv_hbm_gather_probe(const void *buf, size_t chunk_bytes, 
         pkv_set_last_error("hbm_gather_probe: buf must be 16-byte, order and sink 4-byte aligned");
         return PKV_ERR_MISALIGNED;
     }
-    hbm_gather_probe_kernel<<<(unsigned)grid, kProbeThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4 *>(buf), order, n_chunks, (int64_t)(chunk_bytes / 16), sink);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(hbm_gather_probe_kernel, (unsigned)grid, stream, static_cast<const uint4 *>(buf),
+                                     order, n_chunks, (int64_t)(chunk_bytes / 16), sink);
     if (e != cudaSuccess) {
         pkv_set_last_error(cudaGetErrorString(e));
         return PKV_ERR_CUDA;
@@ -127,9 +148,8 @@ extern "C" pkv_status pkv_hbm_read_probe(const void *buf, size_t bytes, unsigned
         pkv_set_last_error("hbm_read_probe: buf must be 16-byte and sink 4-byte aligned");
         return PKV_ERR_MISALIGNED;
     }
-    hbm_read_probe_kernel<<<(unsigned)grid, kProbeThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<const uint4 *>(buf), (int64_t)(bytes / 16), sink);
-    const cudaError_t e = cudaGetLastError();
+    const cudaError_t e = launch_pdl(hbm_read_probe_kernel, (unsigned)grid, stream, static_cast<const uint4 *>(buf),
+                                     (int64_t)(bytes / 16), sink);
     if (e != cudaSuccess) {
         pkv_set_last_error(cudaGetErrorString(e));
         return PKV_ERR_CUDA;
