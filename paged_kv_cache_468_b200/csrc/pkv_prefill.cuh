@@ -127,6 +127,37 @@ enum PfBar {
 // refilled (S_{j+2}) only after P_j V_j has completed: no barrier can run two
 // phases ahead of its waiter.
 
+// Transpose a 4 x 4 array of 16-byte chunks over the four lanes of a quad
+// (q = lane & 3): lane h enters with chunk v of its row in c[v] and leaves
+// with chunk q of quad row h in c[h].  Two exchange stages, with the partner
+// two lanes away and then one lane away; each moves half of the chunks.
+__device__ __forceinline__ uint4 shfl_xor4(const uint4 &x, int m)
+{
+    return make_uint4(__shfl_xor_sync(0xffffffffu, x.x, m), __shfl_xor_sync(0xffffffffu, x.y, m),
+                      __shfl_xor_sync(0xffffffffu, x.z, m), __shfl_xor_sync(0xffffffffu, x.w, m));
+}
+__device__ __forceinline__ void quad_transpose(uint4 (&c)[4], int q)
+{
+    const bool hi = (q & 2) != 0, lo = (q & 1) != 0;
+    uint4 r0 = shfl_xor4(hi ? c[0] : c[2], 2), r1 = shfl_xor4(hi ? c[1] : c[3], 2);
+    if (hi) {
+        c[0] = r0;
+        c[1] = r1;
+    } else {
+        c[2] = r0;
+        c[3] = r1;
+    }
+    r0 = shfl_xor4(lo ? c[0] : c[1], 1);
+    r1 = shfl_xor4(lo ? c[2] : c[3], 1);
+    if (lo) {
+        c[0] = r0;
+        c[2] = r1;
+    } else {
+        c[1] = r0;
+        c[3] = r1;
+    }
+}
+
 // Bits lo .. hi-1 of a 64-column mask (clamped to 0 .. 64; empty when hi <= lo).
 __device__ __forceinline__ uint64_t col_range(int lo, int hi)
 {
@@ -984,6 +1015,16 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         // ---- softmax and epilogue: thread = row r of the tile = TMEM lane r ----
         const int r = warp * 32 + lane;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // row r is (token r / G, head r % G) of the tile; so is the first row
+        // of its quad, r - q.  Divided once here: an integer division goes
+        // through the MUFU unit, which the other softmax warps keep busy.
+        const int q = lane & 3;
+        const int r_tok = r / G, r_head = r - r_tok * G;
+        int rq_tok = r_tok, rq_head = r_head - q;
+        while (rq_head < 0) {
+            rq_head += G;
+            --rq_tok;
+        }
         // for a positive scale the maximum is taken on the raw scores and the
         // scale is folded into the exponent, p = 2^(s*scale - m)
         const float sc = scale_log2;
@@ -996,7 +1037,7 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
         while (ok && next_work(cur)) {
         const int grow = cur.row0 + r;          // row within the sequence
         const bool real = r < R && grow < cur.rows;
-        const int pos = real && MODE == kTcPrefill ? cur.pos0 + r / G : cur.p_max;
+        const int pos = real && MODE == kTcPrefill ? cur.pos0 + r_tok : cur.p_max;
         float m_used = kNegInf;
         float l = 0.f;
         for (int j = 0; j < cur.nt; ++j) {
@@ -1111,23 +1152,50 @@ __device__ __forceinline__ void tc_attend(const CUtensorMap *tm_q, const CUtenso
             const float inv = l > 0.f ? 1.f / l : 0.f;
             // query row (q_tok0 + r / G, head kvh * G + r % G): row0 is a multiple of G
             const size_t orow_i =
-                (size_t)(cur.q_tok0 + r / G) * num_heads + (size_t)cur.kvh * G + r % G;
+                (size_t)(cur.q_tok0 + r_tok) * num_heads + (size_t)cur.kvh * G + r_head;
             if constexpr (MODE == kTcPrefill) {
-                uint4 *orow = reinterpret_cast<uint4 *>(a.out + orow_i * D);
+                // A row is D * 2 contiguous bytes, and rows of different
+                // tokens lie apart.  Each thread normalises its own row, then
+                // the four lanes of a quad trade 16-byte chunks so that a store
+                // instruction writes 64 contiguous bytes of each of eight rows
+                // (one quad per row), not 16 bytes of each of 32 rows.
+                uint4 *orow[4];
+                int tk = rq_tok, hd = rq_head;
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int rr = r - q + h;           // the quad's row h: (token tk, head hd)
+                    const bool rr_real = rr < R && cur.row0 + rr < cur.rows;
+                    orow[h] = rr_real ? reinterpret_cast<uint4 *>(
+                                            a.out + ((size_t)(cur.q_tok0 + tk) * num_heads +
+                                                     (size_t)cur.kvh * G + hd) * D)
+                                      : nullptr;
+                    if (++hd == G) {
+                        hd = 0;
+                        ++tk;
+                    }
+                }
+                // O in two 64-column loads (one for D = 64)
 #pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
-                    uint32_t o[32];
-                    tmem_ld32(tO + lane_base + c0, o);
-                    if (real) {
+                for (int c0 = 0; c0 < D; c0 += 64) {
+                    uint32_t o[64];
+                    tmem_ld64(tO + lane_base + c0, o);
+#pragma unroll
+                    for (int g2 = 0; g2 < 2; ++g2) {
+                        uint4 ch[4];
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
                             uint32_t w[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e)
-                                w[e] = pack2<BF16>(__uint_as_float(o[8 * v + 2 * e]) * inv,
-                                                   __uint_as_float(o[8 * v + 2 * e + 1]) * inv);
-                            orow[c0 / 8 + v] = make_uint4(w[0], w[1], w[2], w[3]);
+                                w[e] = pack2<BF16>(__uint_as_float(o[32 * g2 + 8 * v + 2 * e]) * inv,
+                                                   __uint_as_float(o[32 * g2 + 8 * v + 2 * e + 1]) * inv);
+                            ch[v] = make_uint4(w[0], w[1], w[2], w[3]);
                         }
+                        quad_transpose(ch, q);
+#pragma unroll
+                        for (int h = 0; h < 4; ++h)
+                            if (orow[h] != nullptr)
+                                orow[h][(c0 + 32 * g2) / 8 + q] = ch[h];
                     }
                 }
             } else {

@@ -134,3 +134,14 @@ def test_prefill_many_work_tiles_per_cta():
     step, q, qs = _case(lens, chunks, 16, 4, 128, 16, "bf16", seed=13)
     step["value_cache"] = (step["value_cache"].float() * 0.5).to(torch.bfloat16)
     _check(step, q, qs, chunks)
+
+
+@pytest.mark.parametrize("D,bs,dtype", [(128, 32, "bf16"), (64, 16, "f16")])
+def test_prefill_long_context(D, bs, dtype):
+    """Chunks at the end of contexts of 9000 and 20000 tokens: each row tile
+    walks 140 to 313 key tiles, so every ring and barrier of the pipeline
+    wraps its phase many times within one tile, and the running maximum and
+    sum carry over hundreds of tiles."""
+    lens, chunks = [20000, 9000], [48, 100]
+    step, q, qs = _case(lens, chunks, 4, 1, D, bs, dtype, seed=D + 3)
+    _check(step, q, qs, chunks)
