@@ -145,3 +145,40 @@ def test_prefill_long_context(D, bs, dtype):
     lens, chunks = [20000, 9000], [48, 100]
     step, q, qs = _case(lens, chunks, 4, 1, D, bs, dtype, seed=D + 3)
     _check(step, q, qs, chunks)
+
+
+@pytest.mark.parametrize("name", ["llama3_8b_gqa", "llama13b_mha"])
+def test_prefill_full_size_sampled(name):
+    """The prefill timed by the benchmark (`--op prefill`, chunks of 512): the
+    full workload, its inputs drawn the same way, in one launch with the grid
+    the benchmark gets (several row tiles per CTA on the 8B shape).  The fp64
+    oracle checks a sample of it: the first, last, longest and shortest
+    sequences, and the first and last kv head with their query heads, which
+    attend independently of the other heads."""
+    from paged_kv_cache_468_b200 import workloads
+    cfg = workloads.CONFIGS[name]
+    step = workloads.make_decode_step(cfg)
+    lens = [int(x) for x in step["context_lens"]]
+    chunks = [min(512, L) for L in lens]
+    _, Hq, D = step["query"].shape
+    Hkv = step["key_cache"].shape[2]
+    G = Hq // Hkv
+    g = torch.Generator().manual_seed(cfg.seed + 7)
+    q = torch.randn(sum(chunks), Hq, D, generator=g).to(step["query"].dtype)
+    qs = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    out = pkv.paged_attention_prefill(q.cuda(), torch.from_numpy(qs).cuda(), max(chunks),
+                                      step["key_cache"].cuda(), step["value_cache"].cuda(),
+                                      step["block_tables"].cuda(), step["context_lens"].cuda(),
+                                      step["scale"]).cpu()
+    B = len(lens)
+    seqs = sorted({0, B - 1, int(np.argmax(lens)), int(np.argmin(lens))})
+    kvh = [0, Hkv - 1]
+    qh = [h * G + i for h in kvh for i in range(G)]
+    rows = np.concatenate([np.arange(qs[b], qs[b + 1]) for b in seqs])
+    sub_qs = np.concatenate([[0], np.cumsum([chunks[b] for b in seqs])]).astype(np.int32)
+    ref = oracle.paged_attention_prefill(
+        u16(q[rows][:, qh]), sub_qs, u16(step["key_cache"][:, :, kvh]),
+        u16(step["value_cache"][:, :, kvh]), step["block_tables"].numpy()[seqs],
+        step["context_lens"].numpy()[seqs], step["scale"], step["dtype"], nthreads=NTHREADS)
+    err, idx, finite = max_abs_err(out[rows][:, qh], ref)
+    assert finite and err <= TOL[step["dtype"]], (err, idx)
